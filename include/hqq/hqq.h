@@ -1,0 +1,202 @@
+/*
+ * hqq.h - C ABI of the calibration-free HQQ (Half-Quadratic Quantization) weight
+ * quantize / dequantize path, written for NVIDIA B200 (sm_100a).
+ *
+ * What the operation is (sources, by page title and section):
+ *   - "HQQ calibration-free guide" (lnwmold.com) §2.1: HQQ needs no calibration data; it
+ *     splits the hard, non-convex quantization problem into two simpler sub-problems that
+ *     are solved alternately through an auxiliary variable.
+ *   - same page §2.2: nbits in {8,4,3,2,1}; group_size = weights per group sharing one
+ *     scale/zero; axis selects the direction groups run along a [out_features,in_features]
+ *     weight.
+ *   - same page §3.2: a quantized layer keeps packed low-bit weights (`unpack(dtype=uint8)`)
+ *     and can `dequantize()` back to the compute dtype.
+ *   - "hqq-quantization skill summary" (nav.superapi.store), usage paragraph: the results
+ *     of quantization are W_q, scale and zero, and dequantize() reconstructs W.
+ *   - "HQQ tutorial" (devpress.csdn.net) §3.3: quant_zero / quant_scale quantize the zero
+ *     and scale themselves with a higher precision such as 8 bits.
+ * The pages print no solver formula. The solver computed here is the plainest reading of
+ * their description, written out in full in the comment on hqq_quantize below.
+ *
+ * Conventions for every entry point
+ *   Ownership  The caller owns every buffer. Nothing here allocates, frees or synchronises
+ *              device memory or streams; all device work is enqueued on `stream`.
+ *   Pointers   Arguments documented "device" must be device (or managed) memory on the
+ *              current device. Host pointers there are undefined behaviour.
+ *   Errors     Argument errors are returned synchronously before any launch, and nothing
+ *              is written. A failed launch returns HQQ_ERR_CUDA (the CUDA error string is
+ *              available from hqq_last_cuda_error()). Nothing throws across this ABI.
+ *   Threads    All entry points are re-entrant. hqq_last_cuda_error() is thread-local.
+ *
+ * Packed code layout (fixed here; the pages fix none)
+ *   Group order g:  axis=1: g = r*(cols/gs) + cb, group elements W[r, cb*gs + j]
+ *                   axis=0: g = rb*cols + c,      group elements W[rb*gs + j, c]
+ *   scale/zero are arrays of n_groups values in g order (row-major [rows, cols/gs] for
+ *   axis=1, [rows/gs, cols] for axis=0).
+ *   Code stream:    code k = g*gs + j (row-major W order for axis=1).
+ *     nbits 8,4,2,1: code k sits in byte k/(8/nbits), bits [(k%(8/nbits))*nbits, +nbits),
+ *                    least significant first.
+ *     nbits 3:       code k sits in the little-endian 32-bit word k/10, bits [(k%10)*3, +3);
+ *                    bits 30..31 and unused tail slots are zero.
+ *   Second level (quant_scale / quant_zero): the n_groups meta values, in g order, are cut
+ *   into runs of meta_group_size consecutive values (the last run may be short). Each run
+ *   has uint8 codes and one fp32 pair (step2, zero2), stored interleaved as
+ *   mm[2*i] = step2, mm[2*i+1] = zero2.
+ */
+#ifndef HQQ_HQQ_H_
+#define HQQ_HQQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HQQ_ABI_VERSION 1
+
+typedef enum {
+  HQQ_OK = 0,
+  HQQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, p/beta0/kappa out of range */
+  HQQ_ERR_UNSUPPORTED = 2, /* nbits, group_size, axis or dtype outside the supported set */
+  HQQ_ERR_SHAPE = 3,       /* grouped dimension not divisible by group_size, or too large */
+  HQQ_ERR_ALIGNMENT = 4,   /* a pointer is not aligned as documented */
+  HQQ_ERR_CUDA = 5,        /* a CUDA launch or runtime call failed */
+  HQQ_ERR_WORKSPACE = 6    /* workspace missing or smaller than hqq_workspace_bytes() */
+} hqq_status;
+
+typedef enum { HQQ_F16 = 0, HQQ_BF16 = 1, HQQ_F32 = 2, HQQ_U8 = 3 } hqq_dtype;
+
+/* Supported set (checked on every call):
+ *   nbits       1, 2, 3, 4, 8
+ *   group_size  8, 16, 32, 64, 128, 256
+ *   axis        0 or 1
+ *   iters       0 .. HQQ_MAX_ITERS
+ *   p           0 < p <= 1;  beta0 > 0 and finite;  kappa >= 1 and finite
+ *   W dtype     HQQ_F16, HQQ_BF16, HQQ_F32;  meta dtype HQQ_F16, HQQ_BF16, HQQ_F32
+ *   meta_group_size (second level) 8 .. 1024 */
+#define HQQ_MAX_ITERS 1000
+
+/* Quantization parameters; mirrors BaseQuantizeConfig(nbits, group_size, quant_zero,
+ * quant_scale, axis) of the "HQQ tutorial" (devpress.csdn.net) §3.3, plus the solver
+ * constants p (lp exponent), beta0 (initial penalty) and kappa (penalty growth). */
+typedef struct {
+  int nbits;
+  int group_size;
+  int axis;
+  int iters;
+  float p;
+  float beta0;
+  float kappa;
+  hqq_dtype w_dtype;    /* dtype of W (input of quantize) */
+  hqq_dtype meta_dtype; /* dtype of first-level scale/zero when they are not quantized */
+  int quant_scale;      /* nonzero: scale is stored as uint8 codes + fp32 (step2, zero2) */
+  int quant_zero;       /* nonzero: zero is stored as uint8 codes + fp32 (step2, zero2) */
+  int meta_group_size;  /* run length of the second level (128 in the shipped workloads) */
+} hqq_params;
+
+/* Number of quantization groups of a [rows, cols] weight: rows*cols/group_size.
+ * Returns -1 if the grouped dimension (cols for axis=1, rows for axis=0) is not a multiple
+ * of group_size or an argument is out of range. Host only; no CUDA call. */
+int64_t hqq_num_groups(int64_t rows, int64_t cols, int group_size, int axis);
+
+/* Bytes of the packed code stream for rows*cols codes (layout above):
+ * ceil(N*nbits/8) for nbits 8,4,2,1 and 4*ceil(N/10) for nbits 3. Returns 0 for an
+ * unsupported nbits or a negative size. Host only. */
+size_t hqq_packed_bytes(int64_t rows, int64_t cols, int nbits, int group_size, int axis);
+
+/* Number of second-level runs for n meta values: ceil(n / meta_group_size). Host only. */
+int64_t hqq_num_meta_groups(int64_t n, int meta_group_size);
+
+/* Device workspace hqq_quantize_ex needs for these arguments, in bytes (0 when neither
+ * quant_scale nor quant_zero is set). Host only. Returns (size_t)-1 on invalid params. */
+size_t hqq_workspace_bytes(int64_t rows, int64_t cols, const hqq_params* params);
+
+/* Quantize one weight matrix with the HQQ solver.
+ *
+ * Per group of gs weights w_0..w_{gs-1} (upcast to fp32), with qmax = 2^nbits - 1:
+ *   1. min/max round-to-nearest init: mn, mx; s = qmax/(mx-mn), step = (mx-mn)/qmax
+ *      (s = step = 1 when mx == mn); z = -mn*s; Ws_j = w_j*s.
+ *   2. iters+1 evaluations k = 0..iters of the candidate zero z_k (z_0 is the RTN zero):
+ *      codes Q_j = clamp(rint(Ws_j + z_k), 0, qmax) (round half to even), residual
+ *      r_j = w_j - (Q_j - z_k)*step, lp error e_k = sum_j |r_j|^p. The first candidate
+ *      with the smallest e_k is kept (best-error tracking).
+ *   3. after evaluations 0..iters-1, the auxiliary error variable is the lp generalised
+ *      soft-threshold of the residual, We_j = sign(r_j)*max(|r_j| - |r_j|^(p-1)/beta_k, 0),
+ *      the zero is updated in closed form as a group mean,
+ *      z_{k+1} = mean_j(Q_j - Ws_j + s*We_j), and beta_{k+1} = beta_k*kappa (beta_0 = beta0).
+ *   4. final codes Q*_j = clamp(rint(Ws_j + z_best), 0, qmax); scale = step; zero = z_best.
+ *   Dequantization is then W'_j = (Q*_j - zero)*scale.
+ * Sources: auxiliary variable and alternating minimisation, "HQQ calibration-free guide"
+ * (lnwmold.com) §2.1 and "Dropbox HQQ analysis" (ainews.cool), technical deep dive; a
+ * loss that is lenient on small errors and protects outliers, "HQQ tutorial"
+ * (devpress.csdn.net) §2. The exact steps above are this library's reading of those
+ * passages (the pages give no equations).
+ *
+ * W          device, row-major [rows, cols] of `dtype` (F16, BF16 or F32), 16-byte aligned.
+ * Wq_packed  device, hqq_packed_bytes(...) bytes, 16-byte aligned; fully overwritten.
+ * scale,zero device, n_groups values each of `dtype` (meta dtype = W dtype), naturally
+ *            aligned; written in g order.
+ * Requires cols % group_size == 0 (axis=1) or rows % group_size == 0 (axis=0), and
+ * rows*cols < 2^40. The result is deterministic (bitwise identical run to run). */
+hqq_status hqq_quantize(const void* W, hqq_dtype dtype, int64_t rows, int64_t cols, int nbits,
+                        int group_size, int axis, int iters, float p, float beta0, float kappa,
+                        void* Wq_packed, void* scale, void* zero, cudaStream_t stream);
+
+/* Dequantize: W_out[...] = (float(Q) - zero)*scale in fp32, rounded once (to nearest even)
+ * to `out_dtype`. ("HQQ calibration-free guide" (lnwmold.com) §3.2, dequantize().)
+ * Wq_packed  device, layout above. scale, zero: device, n_groups values of `meta_dtype`.
+ * W_out      device, row-major [rows, cols] of out_dtype (F16, BF16, F32), 16-byte aligned. */
+hqq_status hqq_dequantize(const void* Wq_packed, const void* scale, const void* zero,
+                          hqq_dtype meta_dtype, hqq_dtype out_dtype, int64_t rows, int64_t cols,
+                          int nbits, int group_size, int axis, void* W_out, cudaStream_t stream);
+
+/* Quantize with the full parameter set, including the second level of the "HQQ tutorial"
+ * (devpress.csdn.net) §3.3 (quant_scale / quant_zero: 8-bit min/max round-to-nearest of
+ * the fp32 scale and zero values, runs of meta_group_size values in g order).
+ * scale      device. quant_scale == 0: n_groups values of params->meta_dtype.
+ *                    quant_scale != 0: n_groups uint8 codes.
+ * zero       device, likewise with quant_zero.
+ * scale_mm   device fp32 [n_meta_groups][2] (step2, zero2) when quant_scale, else ignored.
+ * zero_mm    device fp32 [n_meta_groups][2] when quant_zero, else ignored.
+ * workspace  device, >= hqq_workspace_bytes(...) bytes, 16-byte aligned (may be NULL when
+ *            that size is 0). Its contents on entry do not matter and on exit are undefined.
+ *            Two calls that use the same workspace concurrently race. */
+hqq_status hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, const hqq_params* params,
+                           void* Wq_packed, void* scale, void* zero, void* scale_mm, void* zero_mm,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Inverse of hqq_quantize_ex. When quant_scale (quant_zero) is set, the scale (zero) of each
+ * group is first rebuilt in fp32 as (code - zero2)*step2 of its run, and that fp32 value is
+ * used directly. W_out as in hqq_dequantize. */
+hqq_status hqq_dequantize_ex(const void* Wq_packed, const void* scale, const void* zero,
+                             const void* scale_mm, const void* zero_mm, int64_t rows, int64_t cols,
+                             const hqq_params* params, hqq_dtype out_dtype, void* W_out,
+                             cudaStream_t stream);
+
+/* Second level on its own: 8-bit min/max round-to-nearest of n fp32/f16/bf16 values `meta`
+ * (device) in runs of `group` values ("HQQ tutorial" (devpress.csdn.net) §3.3). Per run:
+ * step2 = (max-min)/255, s2 = 255/(max-min) (both 1 when max == min), zero2 = -min*s2,
+ * q = clamp(rint(m*s2 + zero2), 0, 255). q_u8: device, n bytes. mm: device fp32 [runs][2]. */
+hqq_status hqq_quantize_meta(const void* meta, hqq_dtype dtype, int64_t n, int group, void* q_u8,
+                             void* mm, cudaStream_t stream);
+
+/* out_f32[i] = (q_u8[i] - zero2)*step2 of its run, in fp32. All pointers device. */
+hqq_status hqq_dequantize_meta(const void* q_u8, const void* mm, int64_t n, int group,
+                               void* out_f32, cudaStream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* hqq_status_string(hqq_status status);
+
+/* Message of the last CUDA error seen by this thread inside the library ("" if none). */
+const char* hqq_last_cuda_error(void);
+
+/* HQQ_ABI_VERSION of the loaded library. */
+int hqq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQQ_HQQ_H_ */
