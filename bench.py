@@ -1,0 +1,392 @@
+"""Benchmark: whole Llama-7B-shaped model HQQ quantization on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
+
+A step is one pass of the whole hot path over the model: quantize all 224 linear weights
+(32 blocks x q,k,v,o [4096,4096], gate,up [11008,4096], down [4096,11008]; 6,476,005,376 bf16
+weights, 4-bit, group 64, axis 1, iters 20, p 0.7, beta0 10, kappa 1.01) and dequantize
+them all back to bf16. Inputs are synthetic (seeded, LLM-like; see
+calibration_free_weight_hqq_b200/synthetic.py), resident in HBM (13 GB, far above the 126 MB
+L2, so no flush is needed between steps).
+
+Printed on rank 0: one JSON line with the metric (Gweights/s, whole job), the per-kernel
+roofline of the dominant kernel (the solver, bound by the MUFU rate), an end-to-end figure
+through the public API with host buffers, the oracle timed on the host as the CPU baseline,
+and the SM clocks sampled during the timed region.
+
+--impl reference times the CPU oracle (the only reference this path has) on bounded samples
+of the same workload and prints the same metric with "impl": "reference".
+
+Multi-GPU (torchrun): weak scaling - every rank quantizes its own model replica (distinct
+seeds); no collective on the data path; the barrier and the max-over-ranks time use NCCL.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+METRIC = "HQQ quantize Gweights/s & % roofline (HBM|SFU), 7B-shaped bf16 4-bit g64"
+UNIT = "Gweights/s"
+MUFU_PER_CLK_PER_SM = 16          # lg2/ex2 issue rate of the B200 SFU (probed: 15.9)
+N_SM = 148
+SM_MAX_MHZ = 1965.0
+
+
+def peaks():
+    p = {"hbm_gbs": 6535.7, "sm_max_mhz": SM_MAX_MHZ, "source": "fallback"}
+    path = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        p.update({k: m[k] for k in ("hbm_gbs", "sm_max_mhz") if k in m})
+        p["source"] = "measured"
+    return p
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9 or not f[1].isdigit():
+                    continue
+                sm.append(int(f[1]))
+                mx.append(int(f[2]))
+                for n, v in zip(names, f[5:9]):
+                    if v.lower() in ("active", "1"):
+                        reasons.add(n)
+        finally:
+            os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def build_model(workload, device, seed_offset: int):
+    from calibration_free_weight_hqq_b200 import synthetic
+    Ws = []
+    for m in workload.matrices:
+        sigma = synthetic.layer_sigma(m.seed + seed_offset) if m.per_layer_sigma else 0.02
+        Ws.append(synthetic.weight(m.rows, m.cols, seed=m.seed + seed_offset, dtype=m.dtype,
+                                   outlier_rate=m.outlier_rate, sigma_layer=sigma, device=device))
+    return Ws
+
+
+def alloc_outputs(hqq, workload, device):
+    outs, deqs = [], []
+    for m in workload.matrices:
+        ng = m.rows * m.cols // m.group_size
+        outs.append((torch.empty(hqq.hqq_packed_bytes(m.rows, m.cols, m.nbits), dtype=torch.uint8,
+                                 device=device),
+                     torch.empty(ng, dtype=m.dtype, device=device),
+                     torch.empty(ng, dtype=m.dtype, device=device)))
+        deqs.append(torch.empty((m.rows, m.cols), dtype=m.dtype, device=device))
+    return outs, deqs
+
+
+def run_ours(args, rank, world, dev):
+    import calibration_free_weight_hqq_b200 as hqq
+    from calibration_free_weight_hqq_b200 import workloads
+    wl = workloads.llama7b_model_4b()
+    mats = wl.matrices
+    Ws = build_model(wl, dev, seed_offset=rank * 100003)
+    outs, deqs = alloc_outputs(hqq, wl, dev)
+    stream = torch.cuda.current_stream()
+    n_w = wl.weights
+    pk = peaks()
+
+    def step(ev=None):
+        for i, (m, W, (p, s, z)) in enumerate(zip(mats, Ws, outs)):
+            if ev is not None:
+                ev[i][0].record(stream)
+            hqq.hqq_quantize(W, m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0, m.kappa,
+                             Wq_packed=p, scale=s, zero=z, stream=stream)
+            if ev is not None:
+                ev[i][1].record(stream)
+        for m, (p, s, z), D in zip(mats, outs, deqs):
+            hqq.hqq_dequantize(p, s, z, m.rows, m.cols, m.nbits, m.group_size, m.axis,
+                               out=D, stream=stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in mats]
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        barrier()
+        t0.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        t1.record(stream)
+        barrier()
+    ms_total = t0.elapsed_time(t1)
+    q_ms = [e[0].elapsed_time(e[1]) for ev in evs for e in ev]
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = world * n_w / (ms_step * 1e-3) / 1e9
+
+    # roofline of the dominant kernel (the solver): algorithmic MUFU work per launch over
+    # its measured average launch duration
+    launches = len(q_ms)
+    avg_launch_ms = sum(q_ms) / launches
+    mufu_per_weight = 2 * (mats[0].iters + 1)
+    avg_weights = n_w / len(mats)
+    achieved = mufu_per_weight * avg_weights / (avg_launch_ms * 1e-3) / 1e12
+    peak = MUFU_PER_CLK_PER_SM * N_SM * pk["sm_max_mhz"] * 1e6 / 1e12
+    traffic = _traffic_per_launch(avg_weights)
+    clocks = clk.summary()
+    quant_share = sum(q_ms) / args.steps / ms_step
+
+    res = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded LLM-like bf16 weights: per-row sigma, 0.1% outliers)",
+        "config": {"workload": wl.name, "matrices": len(mats), "weights": n_w,
+                   "w_dtype": "bf16", "nbits": 4, "group_size": 64, "axis": 1, "iters": 20,
+                   "p": 0.7, "beta0": 10.0, "kappa": 1.01,
+                   "step": "quantize all 224 matrices + dequantize all 224 to bf16",
+                   "l2": "inputs 13 GB > 126 MB L2, no flush",
+                   "quantize_share_of_step": round(quant_share, 4),
+                   "quantize_Gweights_per_s": round(n_w / (sum(q_ms) / args.steps * 1e-3) / 1e9, 3)},
+        "roofline": {"bound": "alu", "kernel": "quantize_kernel (MUFU lg2+ex2)",
+                     "achieved": round(achieved, 4), "peak": round(peak, 4), "unit": "Top/s (MUFU)",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic": f"{mufu_per_weight} MUFU/weight x {avg_weights:.0f} weights/launch",
+                     "avg_launch_ms": round(avg_launch_ms, 4),
+                     "hbm_frac": round(2.5625 * avg_weights / (avg_launch_ms * 1e-3) / 1e9
+                                       / pk["hbm_gbs"], 4),
+                     "peak_source": f"16 MUFU/clk/SM x 148 SM x {pk['sm_max_mhz']} MHz "
+                                    f"(probed 15.9/clk/SM); hbm {pk['hbm_gbs']} GB/s {pk['source']}"},
+        "clocks": clocks,
+        "gpu_launches": 2 * len(mats) * args.steps,
+    }
+    if rank == 0 and not args.no_e2e:
+        res["e2e"] = run_e2e(hqq, wl, Ws, outs, dev, args)
+    if rank == 0 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl, Ws, args.cpu_seconds)
+    return res
+
+
+def _traffic_per_launch(avg_weights):
+    """DRAM bytes of one solver launch, from the committed ncu capture (bytes per weight
+    measured on a [16384,8192] bf16 launch, scaled to the average launch here); None if no
+    capture of the current kernel is recorded."""
+    path = os.path.join(HERE, "profiles", "quantize_kernel_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    return round(t["dram_bytes_per_weight"] * avg_weights)
+
+
+def run_e2e(hqq, wl, Ws, outs, dev, args):
+    """Same metric through the public API with host buffers: every step copies each weight
+    from pinned host memory, quantizes and dequantizes it, and reads the packed codes and
+    scale/zero back into pinned host memory; copies overlap compute on separate streams."""
+    mats = wl.matrices
+    host_W = [torch.empty_like(W, device="cpu", pin_memory=True).copy_(W) for W in Ws]
+    host_out = [tuple(torch.empty_like(t, device="cpu", pin_memory=True) for t in o)
+                for o in outs]
+    comp = torch.cuda.Stream(dev)
+    h2d = torch.cuda.Stream(dev)
+    d2h = torch.cuda.Stream(dev)
+    n_stage = 3
+    big = max(m.rows * m.cols for m in mats)
+    stage = [torch.empty(big, dtype=torch.bfloat16, device=dev) for _ in range(n_stage)]
+    stage_free = [torch.cuda.Event() for _ in range(n_stage)]
+    deq = torch.empty(big, dtype=torch.bfloat16, device=dev)
+    h2d_bytes = sum(W.numel() * W.element_size() for W in host_W)
+    d2h_bytes = sum(sum(t.numel() * t.element_size() for t in o) for o in host_out)
+
+    def step():
+        out_ready = []
+        for i, m in enumerate(mats):
+            b = i % n_stage
+            buf = stage[b][: m.rows * m.cols].view(m.rows, m.cols)
+            h2d.wait_event(stage_free[b])
+            with torch.cuda.stream(h2d):
+                buf.copy_(host_W[i], non_blocking=True)
+                loaded = torch.cuda.Event()
+                loaded.record(h2d)
+            comp.wait_event(loaded)
+            p, s, z = outs[i]
+            hqq.hqq_quantize(buf, m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0, m.kappa,
+                             Wq_packed=p, scale=s, zero=z, stream=comp)
+            hqq.hqq_dequantize(p, s, z, m.rows, m.cols, m.nbits, m.group_size, m.axis,
+                               out=deq[: m.rows * m.cols].view(m.rows, m.cols), stream=comp)
+            stage_free[b].record(comp)
+            done = torch.cuda.Event()
+            done.record(comp)
+            d2h.wait_event(done)
+            with torch.cuda.stream(d2h):
+                for src, dst in zip(outs[i], host_out[i]):
+                    dst.copy_(src, non_blocking=True)
+        d2h.synchronize()
+        comp.synchronize()
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 3))
+    t = time.perf_counter()
+    for _ in range(steps):
+        step()
+    torch.cuda.synchronize()
+    sec = (time.perf_counter() - t) / steps
+    return {"value": round(wl.weights / sec / 1e9, 3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
+            "ms_per_step": round(sec * 1e3, 2), "steps": steps,
+            "how": "pinned host W -> device (stream 1), quantize+dequantize (stream 2), "
+                   "packed+scale+zero -> pinned host (stream 3); wall clock with device sync"}
+
+
+def cpu_baseline(wl, Ws, seconds: float, impl_line=False):
+    """The oracle, as it stands, on the host cores over a bounded sample of the workload:
+    whole row blocks of the model's matrices in order until `seconds` of CPU time."""
+    import oracle
+    nt = oracle.default_threads()
+    done_w, t_used, parts = 0, 0.0, []
+    rows_per = 256
+    i = 0
+    while t_used < seconds and i < len(wl.matrices):
+        m, W = wl.matrices[i], Ws[i]
+        for r0 in range(0, m.rows, rows_per):
+            Wh = W[r0:r0 + rows_per].float().cpu().numpy()
+            t = time.perf_counter()
+            oracle.quantize(Wh, m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0, m.kappa,
+                            nthreads=nt)
+            t_used += time.perf_counter() - t
+            done_w += Wh.size
+            if t_used >= seconds:
+                break
+        parts.append(m.name)
+        i += 1
+    return {"value": round(done_w / t_used / 1e9, 5), "unit": UNIT, "cores": nt, "kind": "oracle",
+            "sample": f"{done_w} weights ({len(parts)} matrices, row blocks of {rows_per}) "
+                      f"in {t_used:.1f} s of oracle time, {nt} threads"}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle on bounded samples, timed per step."""
+    from calibration_free_weight_hqq_b200 import workloads
+    import oracle
+    wl = workloads.llama7b_model_4b()
+    nt = oracle.default_threads()
+    m = wl.matrices[4]  # gate_proj [11008, 4096]
+    from calibration_free_weight_hqq_b200 import synthetic
+    W = synthetic.weight(m.rows, m.cols, seed=m.seed, dtype=m.dtype, outlier_rate=m.outlier_rate,
+                         sigma_layer=synthetic.layer_sigma(m.seed)).float().numpy()
+    rows = max(16, int(os.environ.get("HQQ_REF_ROWS", "512")))
+    sample = W[:rows]
+    for _ in range(args.warmup):
+        oracle.quantize(sample, m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0, m.kappa,
+                        nthreads=nt)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.quantize(sample, m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0, m.kappa,
+                        nthreads=nt)
+    sec = (time.perf_counter() - t) / args.steps
+    value = sample.size / sec / 1e9
+    desc = f"{rows} rows of {m.name} [{m.rows},{m.cols}] ({sample.size} weights) per step"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "sample": desc},
+            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": nt, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        res = run_ours(args, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,265 @@
+"""calibration_free_weight_hqq_b200 - HQQ weight quantize / dequantize on NVIDIA B200.
+
+A thin Python binding over the C ABI of ``libhqq_b200.so`` (declared in
+``include/hqq/hqq.h``). The functions carry the C names and only marshal arguments:
+PyTorch supplies device memory and the current stream, and every step of quantization and
+dequantization runs in the library's CUDA kernels. There is no CPU fallback: if the
+library is missing or the tensors are not on a CUDA device, the calls raise.
+
+    import torch, calibration_free_weight_hqq_b200 as hqq
+    W = torch.randn(4096, 1024, device="cuda", dtype=torch.float16) * 0.02
+    Wq, scale, zero = hqq.hqq_quantize(W, nbits=4, group_size=64, axis=1)
+    W2 = hqq.hqq_dequantize(Wq, scale, zero, 4096, 1024, nbits=4, group_size=64, axis=1,
+                            out_dtype=torch.float16)
+
+Parameters mirror BaseQuantizeConfig(nbits, group_size, quant_zero, quant_scale, axis)
+("HQQ tutorial" (devpress.csdn.net) §3.3) plus the solver constants iters, p, beta0, kappa.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "HQQError", "HQQParams", "lib", "library_path", "hqq_quantize", "hqq_quantize_ex",
+    "hqq_dequantize", "hqq_dequantize_ex", "hqq_quantize_meta", "hqq_dequantize_meta",
+    "hqq_packed_bytes", "hqq_num_groups", "hqq_num_meta_groups", "hqq_workspace_bytes",
+    "HQQ_F16", "HQQ_BF16", "HQQ_F32", "HQQ_U8",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libhqq_b200.so")
+_lock = threading.Lock()
+_lib = None
+
+HQQ_F16, HQQ_BF16, HQQ_F32, HQQ_U8 = 0, 1, 2, 3
+_TORCH_DT = {torch.float16: HQQ_F16, torch.bfloat16: HQQ_BF16, torch.float32: HQQ_F32,
+             torch.uint8: HQQ_U8}
+_DT_TORCH = {v: k for k, v in _TORCH_DT.items()}
+
+
+class HQQError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        name = lib().hqq_status_string(status).decode()
+        super().__init__(f"{where}: {name}" + (f" ({detail})" if detail else ""))
+
+
+class HQQParams(ctypes.Structure):
+    """Mirror of the C struct hqq_params."""
+    _fields_ = [("nbits", ctypes.c_int), ("group_size", ctypes.c_int), ("axis", ctypes.c_int),
+                ("iters", ctypes.c_int), ("p", ctypes.c_float), ("beta0", ctypes.c_float),
+                ("kappa", ctypes.c_float), ("w_dtype", ctypes.c_int),
+                ("meta_dtype", ctypes.c_int), ("quant_scale", ctypes.c_int),
+                ("quant_zero", ctypes.c_int), ("meta_group_size", ctypes.c_int)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is missing: build it with "
+                    "`python -m calibration_free_weight_hqq_b200.build` (nvcc, sm_100a)")
+            L = ctypes.CDLL(_LIB_PATH)
+            P, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+            sz = ctypes.c_size_t
+            L.hqq_quantize.argtypes = [P, i32, i64, i64, i32, i32, i32, i32, f32, f32, f32, P, P,
+                                       P, P]
+            L.hqq_dequantize.argtypes = [P, P, P, i32, i32, i64, i64, i32, i32, i32, P, P]
+            L.hqq_quantize_ex.argtypes = [P, i64, i64, ctypes.POINTER(HQQParams), P, P, P, P, P,
+                                          P, sz, P]
+            L.hqq_dequantize_ex.argtypes = [P, P, P, P, P, i64, i64, ctypes.POINTER(HQQParams),
+                                            i32, P, P]
+            L.hqq_quantize_meta.argtypes = [P, i32, i64, i32, P, P, P]
+            L.hqq_dequantize_meta.argtypes = [P, P, i64, i32, P, P]
+            for f in ("hqq_quantize", "hqq_dequantize", "hqq_quantize_ex", "hqq_dequantize_ex",
+                      "hqq_quantize_meta", "hqq_dequantize_meta"):
+                getattr(L, f).restype = i32
+            L.hqq_packed_bytes.argtypes = [i64, i64, i32, i32, i32]
+            L.hqq_packed_bytes.restype = sz
+            L.hqq_num_groups.argtypes = [i64, i64, i32, i32]
+            L.hqq_num_groups.restype = i64
+            L.hqq_num_meta_groups.argtypes = [i64, i32]
+            L.hqq_num_meta_groups.restype = i64
+            L.hqq_workspace_bytes.argtypes = [i64, i64, ctypes.POINTER(HQQParams)]
+            L.hqq_workspace_bytes.restype = sz
+            L.hqq_status_string.argtypes = [i32]
+            L.hqq_status_string.restype = ctypes.c_char_p
+            L.hqq_last_cuda_error.argtypes = []
+            L.hqq_last_cuda_error.restype = ctypes.c_char_p
+            L.hqq_abi_version.argtypes = []
+            L.hqq_abi_version.restype = i32
+            _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        detail = lib().hqq_last_cuda_error().decode() if status == 5 else ""
+        raise HQQError(status, where, detail)
+
+
+def _cuda(t: torch.Tensor, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def hqq_packed_bytes(rows: int, cols: int, nbits: int, group_size: int = 64, axis: int = 1) -> int:
+    return int(lib().hqq_packed_bytes(rows, cols, nbits, group_size, axis))
+
+
+def hqq_num_groups(rows: int, cols: int, group_size: int, axis: int) -> int:
+    return int(lib().hqq_num_groups(rows, cols, group_size, axis))
+
+
+def hqq_num_meta_groups(n: int, meta_group_size: int) -> int:
+    return int(lib().hqq_num_meta_groups(n, meta_group_size))
+
+
+def _meta_shape(rows: int, cols: int, group_size: int, axis: int):
+    return (rows, cols // group_size) if axis == 1 else (rows // group_size, cols)
+
+
+def make_params(nbits=4, group_size=64, axis=1, iters=20, p=0.7, beta0=10.0, kappa=1.01,
+                w_dtype=torch.bfloat16, meta_dtype=None, quant_scale=False, quant_zero=False,
+                meta_group_size=128) -> HQQParams:
+    meta_dtype = w_dtype if meta_dtype is None else meta_dtype
+    return HQQParams(nbits, group_size, axis, iters, p, beta0, kappa, _TORCH_DT[w_dtype],
+                     _TORCH_DT[meta_dtype], int(bool(quant_scale)), int(bool(quant_zero)),
+                     meta_group_size)
+
+
+def hqq_workspace_bytes(rows: int, cols: int, params: HQQParams) -> int:
+    n = lib().hqq_workspace_bytes(rows, cols, ctypes.byref(params))
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid parameters")
+    return int(n)
+
+
+def hqq_quantize(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: int = 1,
+                 iters: int = 20, p: float = 0.7, beta0: float = 10.0, kappa: float = 1.01, *,
+                 Wq_packed: Optional[torch.Tensor] = None, scale: Optional[torch.Tensor] = None,
+                 zero: Optional[torch.Tensor] = None, stream=None):
+    """Quantize a 2-D CUDA weight (fp16/bf16/fp32). Returns (Wq_packed uint8, scale, zero),
+    scale/zero in W's dtype, shaped [rows, cols/G] (axis=1) or [rows/G, cols] (axis=0)."""
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [out_features, in_features]")
+    rows, cols = W.shape
+    wp = _cuda(W, "W")
+    if Wq_packed is None:
+        Wq_packed = torch.empty(hqq_packed_bytes(rows, cols, nbits, group_size, axis),
+                                dtype=torch.uint8, device=W.device)
+    ms = _meta_shape(rows, cols, group_size, axis) if hqq_num_groups(rows, cols, group_size, axis) >= 0 else (0,)
+    if scale is None:
+        scale = torch.empty(ms, dtype=W.dtype, device=W.device)
+    if zero is None:
+        zero = torch.empty(ms, dtype=W.dtype, device=W.device)
+    st = lib().hqq_quantize(wp, _TORCH_DT.get(W.dtype, -1), rows, cols, nbits, group_size, axis,
+                            iters, p, beta0, kappa, _cuda(Wq_packed, "Wq_packed"),
+                            _cuda(scale, "scale"), _cuda(zero, "zero"), _stream(stream))
+    _check(st, "hqq_quantize")
+    return Wq_packed, scale, zero
+
+
+def hqq_quantize_ex(W: torch.Tensor, params: HQQParams, *, stream=None, workspace=None):
+    """Full parameter set (second-level 8-bit scale/zero). Returns a dict with Wq_packed,
+    scale, zero (uint8 codes when quantized) and scale_mm / zero_mm (fp32 [runs, 2])."""
+    rows, cols = W.shape
+    wp = _cuda(W, "W")
+    dev = W.device
+    ng = hqq_num_groups(rows, cols, params.group_size, params.axis)
+    if ng < 0:
+        raise HQQError(3, "hqq_quantize_ex")
+    ms = _meta_shape(rows, cols, params.group_size, params.axis)
+    mdt = _DT_TORCH[params.meta_dtype]
+    runs = max(hqq_num_meta_groups(ng, params.meta_group_size), 0)
+    out = {
+        "Wq_packed": torch.empty(hqq_packed_bytes(rows, cols, params.nbits), dtype=torch.uint8,
+                                 device=dev),
+        "scale": torch.empty(ms, dtype=torch.uint8 if params.quant_scale else mdt, device=dev),
+        "zero": torch.empty(ms, dtype=torch.uint8 if params.quant_zero else mdt, device=dev),
+        "scale_mm": torch.empty((runs, 2), dtype=torch.float32, device=dev)
+        if params.quant_scale else None,
+        "zero_mm": torch.empty((runs, 2), dtype=torch.float32, device=dev)
+        if params.quant_zero else None,
+    }
+    need = hqq_workspace_bytes(rows, cols, params)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = lib().hqq_quantize_ex(
+        wp, rows, cols, ctypes.byref(params), _cuda(out["Wq_packed"], "Wq_packed"),
+        _cuda(out["scale"], "scale"), _cuda(out["zero"], "zero"),
+        out["scale_mm"].data_ptr() if out["scale_mm"] is not None else None,
+        out["zero_mm"].data_ptr() if out["zero_mm"] is not None else None,
+        workspace.data_ptr() if workspace is not None else None,
+        workspace.numel() if workspace is not None else 0, _stream(stream))
+    _check(st, "hqq_quantize_ex")
+    return out
+
+
+def hqq_dequantize(Wq_packed, scale, zero, rows: int, cols: int, nbits: int = 4,
+                   group_size: int = 64, axis: int = 1, out_dtype=torch.bfloat16, *, out=None,
+                   stream=None):
+    """Dequantize to a [rows, cols] CUDA tensor of out_dtype."""
+    if out is None:
+        out = torch.empty((rows, cols), dtype=out_dtype, device=Wq_packed.device)
+    st = lib().hqq_dequantize(_cuda(Wq_packed, "Wq_packed"), _cuda(scale, "scale"),
+                              _cuda(zero, "zero"), _TORCH_DT.get(scale.dtype, -1),
+                              _TORCH_DT.get(out.dtype, -1), rows, cols, nbits, group_size, axis,
+                              _cuda(out, "out"), _stream(stream))
+    _check(st, "hqq_dequantize")
+    return out
+
+
+def hqq_dequantize_ex(q: dict, rows: int, cols: int, params: HQQParams, out_dtype=torch.bfloat16,
+                      *, out=None, stream=None):
+    """Inverse of hqq_quantize_ex (q is its result dict)."""
+    if out is None:
+        out = torch.empty((rows, cols), dtype=out_dtype, device=q["Wq_packed"].device)
+    smm, zmm = q.get("scale_mm"), q.get("zero_mm")
+    st = lib().hqq_dequantize_ex(
+        _cuda(q["Wq_packed"], "Wq_packed"), _cuda(q["scale"], "scale"), _cuda(q["zero"], "zero"),
+        smm.data_ptr() if smm is not None else None, zmm.data_ptr() if zmm is not None else None,
+        rows, cols, ctypes.byref(params), _TORCH_DT.get(out.dtype, -1), _cuda(out, "out"),
+        _stream(stream))
+    _check(st, "hqq_dequantize_ex")
+    return out
+
+
+def hqq_quantize_meta(meta: torch.Tensor, group: int = 128, *, stream=None):
+    """Second level alone: returns (uint8 codes [n], fp32 [runs, 2] (step2, zero2))."""
+    n = meta.numel()
+    q = torch.empty(n, dtype=torch.uint8, device=meta.device)
+    mm = torch.empty((max(hqq_num_meta_groups(n, group), 0), 2), dtype=torch.float32,
+                     device=meta.device)
+    st = lib().hqq_quantize_meta(_cuda(meta, "meta"), _TORCH_DT.get(meta.dtype, -1), n, group,
+                                 _cuda(q, "q"), _cuda(mm, "mm"), _stream(stream))
+    _check(st, "hqq_quantize_meta")
+    return q, mm
+
+
+def hqq_dequantize_meta(q: torch.Tensor, mm: torch.Tensor, group: int = 128, *, stream=None):
+    out = torch.empty(q.numel(), dtype=torch.float32, device=q.device)
+    st = lib().hqq_dequantize_meta(_cuda(q, "q"), _cuda(mm, "mm"), q.numel(), group,
+                                   _cuda(out, "out"), _stream(stream))
+    _check(st, "hqq_dequantize_meta")
+    return out

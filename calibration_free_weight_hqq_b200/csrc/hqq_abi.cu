@@ -1,0 +1,290 @@
+// hqq_abi.cu - extern "C" entry points of libhqq_b200.so: argument validation (pure host
+// arithmetic, no CUDA call before the arguments are known to be valid) and dispatch to the
+// kernels. Declarations and the full contract are in include/hqq/hqq.h.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/hqq/hqq.h"
+#include "hqq_kernels.h"
+
+#define HQQ_EXPORT extern "C" __attribute__((visibility("default")))
+
+static_assert((int)HQQ_F16 == hqqk::kF16 && (int)HQQ_BF16 == hqqk::kBF16 &&
+                  (int)HQQ_F32 == hqqk::kF32 && (int)HQQ_U8 == hqqk::kU8,
+              "dtype enumerators must match");
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+hqq_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return HQQ_OK;
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return HQQ_ERR_CUDA;
+}
+
+constexpr int64_t kMaxElems = int64_t(1) << 40;
+
+bool nbits_ok(int nbits) {
+  return nbits == 1 || nbits == 2 || nbits == 3 || nbits == 4 || nbits == 8;
+}
+bool group_ok(int g) { return g == 8 || g == 16 || g == 32 || g == 64 || g == 128 || g == 256; }
+bool wdtype_ok(int dt) { return dt == HQQ_F16 || dt == HQQ_BF16 || dt == HQQ_F32; }
+size_t dtype_size(int dt) { return dt == HQQ_F32 ? 4 : dt == HQQ_U8 ? 1 : 2; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape checks shared by quantize and dequantize.
+hqq_status check_shape(int64_t rows, int64_t cols, int nbits, int group_size, int axis) {
+  if (rows < 0 || cols < 0) return HQQ_ERR_INVALID_ARG;
+  if (!nbits_ok(nbits) || !group_ok(group_size) || (axis != 0 && axis != 1))
+    return HQQ_ERR_UNSUPPORTED;
+  if (cols > 0 && rows > kMaxElems / cols) return HQQ_ERR_SHAPE;
+  if (axis == 1 && cols % group_size) return HQQ_ERR_SHAPE;
+  if (axis == 0 && rows % group_size) return HQQ_ERR_SHAPE;
+  return HQQ_OK;
+}
+
+hqq_status check_solver(int iters, float p, float beta0, float kappa) {
+  if (iters < 0 || iters > HQQ_MAX_ITERS) return HQQ_ERR_INVALID_ARG;
+  if (!(p > 0.0f && p <= 1.0f)) return HQQ_ERR_INVALID_ARG;
+  if (!(beta0 > 0.0f) || !isfinite(beta0)) return HQQ_ERR_INVALID_ARG;
+  if (!(kappa >= 1.0f) || !isfinite(kappa)) return HQQ_ERR_INVALID_ARG;
+  return HQQ_OK;
+}
+
+hqq_status check_meta_group(int g) { return (g >= 8 && g <= 1024) ? HQQ_OK : HQQ_ERR_UNSUPPORTED; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+HQQ_EXPORT int hqq_abi_version(void) { return HQQ_ABI_VERSION; }
+
+HQQ_EXPORT const char* hqq_last_cuda_error(void) { return g_last_cuda_error; }
+
+HQQ_EXPORT const char* hqq_status_string(hqq_status s) {
+  switch (s) {
+    case HQQ_OK: return "HQQ_OK";
+    case HQQ_ERR_INVALID_ARG: return "HQQ_ERR_INVALID_ARG";
+    case HQQ_ERR_UNSUPPORTED: return "HQQ_ERR_UNSUPPORTED";
+    case HQQ_ERR_SHAPE: return "HQQ_ERR_SHAPE";
+    case HQQ_ERR_ALIGNMENT: return "HQQ_ERR_ALIGNMENT";
+    case HQQ_ERR_CUDA: return "HQQ_ERR_CUDA";
+    case HQQ_ERR_WORKSPACE: return "HQQ_ERR_WORKSPACE";
+  }
+  return "HQQ_ERR_UNKNOWN";
+}
+
+HQQ_EXPORT int64_t hqq_num_groups(int64_t rows, int64_t cols, int group_size, int axis) {
+  if (!group_ok(group_size) || (axis != 0 && axis != 1) || rows < 0 || cols < 0) return -1;
+  if (cols > 0 && rows > kMaxElems / cols) return -1;
+  if (axis == 1 && cols % group_size) return -1;
+  if (axis == 0 && rows % group_size) return -1;
+  return rows * cols / group_size;
+}
+
+HQQ_EXPORT size_t hqq_packed_bytes(int64_t rows, int64_t cols, int nbits, int group_size, int axis) {
+  (void)group_size;
+  (void)axis;
+  if (!nbits_ok(nbits) || rows < 0 || cols < 0) return 0;
+  if (cols > 0 && rows > kMaxElems / cols) return 0;
+  const int64_t n = rows * cols;
+  if (nbits == 3) return (size_t)(4 * ((n + 9) / 10));
+  return (size_t)((n * nbits + 7) / 8);
+}
+
+HQQ_EXPORT int64_t hqq_num_meta_groups(int64_t n, int meta_group_size) {
+  if (n < 0 || meta_group_size <= 0) return -1;
+  return (n + meta_group_size - 1) / meta_group_size;
+}
+
+// Workspace: fp32 scale then fp32 zero (only the quantized ones), each part 256-aligned.
+HQQ_EXPORT size_t hqq_workspace_bytes(int64_t rows, int64_t cols, const hqq_params* prm) {
+  if (!prm) return (size_t)-1;
+  const int64_t ng = hqq_num_groups(rows, cols, prm->group_size, prm->axis);
+  if (ng < 0) return (size_t)-1;
+  const size_t part = round_up((size_t)ng * 4, 256);
+  return part * ((prm->quant_scale ? 1 : 0) + (prm->quant_zero ? 1 : 0));
+}
+
+static hqq_status quantize_impl(const void* W, int64_t rows, int64_t cols, const hqq_params& prm,
+                                void* Wq_packed, void* scale, void* zero, void* scale_mm,
+                                void* zero_mm, void* workspace, size_t workspace_bytes,
+                                cudaStream_t stream) {
+  hqq_status st = check_shape(rows, cols, prm.nbits, prm.group_size, prm.axis);
+  if (st != HQQ_OK) return st;
+  if ((st = check_solver(prm.iters, prm.p, prm.beta0, prm.kappa)) != HQQ_OK) return st;
+  if (!wdtype_ok(prm.w_dtype) || !wdtype_ok(prm.meta_dtype)) return HQQ_ERR_UNSUPPORTED;
+  const bool qs = prm.quant_scale != 0, qz = prm.quant_zero != 0;
+  if ((qs || qz) && (st = check_meta_group(prm.meta_group_size)) != HQQ_OK) return st;
+  if (rows * cols == 0) return HQQ_OK;  // nothing to read or write; pointers may be NULL
+  if (!W || !Wq_packed || !scale || !zero) return HQQ_ERR_INVALID_ARG;
+  if ((qs && !scale_mm) || (qz && !zero_mm)) return HQQ_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(Wq_packed, 16)) return HQQ_ERR_ALIGNMENT;
+  const size_t msz = dtype_size(prm.meta_dtype);
+  if (!qs && !aligned(scale, msz)) return HQQ_ERR_ALIGNMENT;
+  if (!qz && !aligned(zero, msz)) return HQQ_ERR_ALIGNMENT;
+  if ((qs && !aligned(scale_mm, 8)) || (qz && !aligned(zero_mm, 8))) return HQQ_ERR_ALIGNMENT;
+  const size_t need = hqq_workspace_bytes(rows, cols, &prm);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return HQQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return HQQ_ERR_ALIGNMENT;
+  }
+  const int64_t ng = rows * cols / prm.group_size;
+
+  const size_t part = round_up((size_t)ng * 4, 256);
+  float* ws_scale = qs ? reinterpret_cast<float*>(workspace) : nullptr;
+  float* ws_zero = qz ? reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + (qs ? part : 0))
+                      : nullptr;
+
+  hqqk::QuantJob j;
+  j.W = W;
+  j.rows = rows;
+  j.cols = cols;
+  j.n_groups = ng;
+  j.w_dtype = prm.w_dtype;
+  j.nbits = prm.nbits;
+  j.group_size = prm.group_size;
+  j.axis = prm.axis;
+  j.iters = prm.iters;
+  j.p = prm.p;
+  j.beta0 = prm.beta0;
+  j.kappa = prm.kappa;
+  j.packed = reinterpret_cast<uint8_t*>(Wq_packed);
+  j.scale = qs ? static_cast<void*>(ws_scale) : scale;
+  j.zero = qz ? static_cast<void*>(ws_zero) : zero;
+  j.scale_dtype = qs ? hqqk::kF32 : prm.meta_dtype;
+  j.zero_dtype = qz ? hqqk::kF32 : prm.meta_dtype;
+  if ((st = cuda_status(hqqk::launch_quantize(j, stream))) != HQQ_OK) return st;
+  if (qs) {
+    st = cuda_status(hqqk::launch_quantize_meta(ws_scale, hqqk::kF32, ng, prm.meta_group_size,
+                                                reinterpret_cast<uint8_t*>(scale),
+                                                reinterpret_cast<float*>(scale_mm), stream));
+    if (st != HQQ_OK) return st;
+  }
+  if (qz) {
+    st = cuda_status(hqqk::launch_quantize_meta(ws_zero, hqqk::kF32, ng, prm.meta_group_size,
+                                                reinterpret_cast<uint8_t*>(zero),
+                                                reinterpret_cast<float*>(zero_mm), stream));
+    if (st != HQQ_OK) return st;
+  }
+  return HQQ_OK;
+}
+
+HQQ_EXPORT hqq_status hqq_quantize(const void* W, hqq_dtype dtype, int64_t rows, int64_t cols,
+                                   int nbits, int group_size, int axis, int iters, float p,
+                                   float beta0, float kappa, void* Wq_packed, void* scale,
+                                   void* zero, cudaStream_t stream) {
+  hqq_params prm;
+  prm.nbits = nbits;
+  prm.group_size = group_size;
+  prm.axis = axis;
+  prm.iters = iters;
+  prm.p = p;
+  prm.beta0 = beta0;
+  prm.kappa = kappa;
+  prm.w_dtype = dtype;
+  prm.meta_dtype = dtype;
+  prm.quant_scale = 0;
+  prm.quant_zero = 0;
+  prm.meta_group_size = 128;
+  return quantize_impl(W, rows, cols, prm, Wq_packed, scale, zero, nullptr, nullptr, nullptr, 0,
+                       stream);
+}
+
+HQQ_EXPORT hqq_status hqq_quantize_ex(const void* W, int64_t rows, int64_t cols,
+                                      const hqq_params* params, void* Wq_packed, void* scale,
+                                      void* zero, void* scale_mm, void* zero_mm, void* workspace,
+                                      size_t workspace_bytes, cudaStream_t stream) {
+  if (!params) return HQQ_ERR_INVALID_ARG;
+  return quantize_impl(W, rows, cols, *params, Wq_packed, scale, zero, scale_mm, zero_mm,
+                       workspace, workspace_bytes, stream);
+}
+
+static hqq_status dequantize_impl(const void* Wq_packed, const void* scale, const void* zero,
+                                  const void* scale_mm, const void* zero_mm, int meta_dtype,
+                                  int meta_group_size, int64_t rows, int64_t cols, int nbits,
+                                  int group_size, int axis, int out_dtype, void* W_out,
+                                  cudaStream_t stream) {
+  hqq_status st = check_shape(rows, cols, nbits, group_size, axis);
+  if (st != HQQ_OK) return st;
+  if (!wdtype_ok(out_dtype)) return HQQ_ERR_UNSUPPORTED;
+  if ((!scale_mm || !zero_mm) && !wdtype_ok(meta_dtype)) return HQQ_ERR_UNSUPPORTED;
+  if ((scale_mm || zero_mm) && (st = check_meta_group(meta_group_size)) != HQQ_OK) return st;
+  if (rows * cols == 0) return HQQ_OK;
+  if (!Wq_packed || !scale || !zero || !W_out) return HQQ_ERR_INVALID_ARG;
+  if (!aligned(Wq_packed, 16) || !aligned(W_out, 16)) return HQQ_ERR_ALIGNMENT;
+  const size_t msz = dtype_size(meta_dtype);
+  if ((!scale_mm && !aligned(scale, msz)) || (!zero_mm && !aligned(zero, msz)))
+    return HQQ_ERR_ALIGNMENT;
+  if ((scale_mm && !aligned(scale_mm, 8)) || (zero_mm && !aligned(zero_mm, 8)))
+    return HQQ_ERR_ALIGNMENT;
+  hqqk::DequantJob j;
+  j.packed = reinterpret_cast<const uint8_t*>(Wq_packed);
+  j.scale = scale;
+  j.zero = zero;
+  j.scale_mm = reinterpret_cast<const float*>(scale_mm);
+  j.zero_mm = reinterpret_cast<const float*>(zero_mm);
+  j.meta_group_size = meta_group_size;
+  j.meta_dtype = meta_dtype;
+  j.rows = rows;
+  j.cols = cols;
+  j.n_groups = rows * cols / group_size;
+  j.nbits = nbits;
+  j.group_size = group_size;
+  j.axis = axis;
+  j.out_dtype = out_dtype;
+  j.out = W_out;
+  return cuda_status(hqqk::launch_dequantize(j, stream));
+}
+
+HQQ_EXPORT hqq_status hqq_dequantize(const void* Wq_packed, const void* scale, const void* zero,
+                                     hqq_dtype meta_dtype, hqq_dtype out_dtype, int64_t rows,
+                                     int64_t cols, int nbits, int group_size, int axis,
+                                     void* W_out, cudaStream_t stream) {
+  return dequantize_impl(Wq_packed, scale, zero, nullptr, nullptr, meta_dtype, 128, rows, cols,
+                         nbits, group_size, axis, out_dtype, W_out, stream);
+}
+
+HQQ_EXPORT hqq_status hqq_dequantize_ex(const void* Wq_packed, const void* scale, const void* zero,
+                                        const void* scale_mm, const void* zero_mm, int64_t rows,
+                                        int64_t cols, const hqq_params* params,
+                                        hqq_dtype out_dtype, void* W_out, cudaStream_t stream) {
+  if (!params) return HQQ_ERR_INVALID_ARG;
+  const void* smm = params->quant_scale ? scale_mm : nullptr;
+  const void* zmm = params->quant_zero ? zero_mm : nullptr;
+  if ((params->quant_scale && !scale_mm) || (params->quant_zero && !zero_mm))
+    return HQQ_ERR_INVALID_ARG;
+  return dequantize_impl(Wq_packed, scale, zero, smm, zmm, params->meta_dtype,
+                         params->meta_group_size, rows, cols, params->nbits, params->group_size,
+                         params->axis, out_dtype, W_out, stream);
+}
+
+HQQ_EXPORT hqq_status hqq_quantize_meta(const void* meta, hqq_dtype dtype, int64_t n, int group,
+                                        void* q_u8, void* mm, cudaStream_t stream) {
+  if (n < 0) return HQQ_ERR_INVALID_ARG;
+  if (!wdtype_ok(dtype)) return HQQ_ERR_UNSUPPORTED;
+  hqq_status st = check_meta_group(group);
+  if (st != HQQ_OK) return st;
+  if (n == 0) return HQQ_OK;
+  if (!meta || !q_u8 || !mm) return HQQ_ERR_INVALID_ARG;
+  if (!aligned(meta, dtype_size(dtype)) || !aligned(mm, 8)) return HQQ_ERR_ALIGNMENT;
+  return cuda_status(hqqk::launch_quantize_meta(meta, dtype, n, group,
+                                                reinterpret_cast<uint8_t*>(q_u8),
+                                                reinterpret_cast<float*>(mm), stream));
+}
+
+HQQ_EXPORT hqq_status hqq_dequantize_meta(const void* q_u8, const void* mm, int64_t n, int group,
+                                          void* out_f32, cudaStream_t stream) {
+  if (n < 0) return HQQ_ERR_INVALID_ARG;
+  hqq_status st = check_meta_group(group);
+  if (st != HQQ_OK) return st;
+  if (n == 0) return HQQ_OK;
+  if (!q_u8 || !mm || !out_f32) return HQQ_ERR_INVALID_ARG;
+  if (!aligned(mm, 8) || !aligned(out_f32, 4)) return HQQ_ERR_ALIGNMENT;
+  return cuda_status(hqqk::launch_dequantize_meta(reinterpret_cast<const uint8_t*>(q_u8),
+                                                  reinterpret_cast<const float*>(mm), n, group,
+                                                  reinterpret_cast<float*>(out_f32), stream));
+}

@@ -1,0 +1,330 @@
+// hqq_dequantize.cu - dequantization and second-level (8-bit meta) kernels for sm_100a.
+//
+// Dequantize ("HQQ calibration-free guide" (lnwmold.com) §3.2, dequantize(); "hqq-quantization
+// skill summary" (nav.superapi.store), usage): W'[i] = (float(Q_i) - zero_g)*scale_g in fp32,
+// two separate roundings, then one rounding to nearest even to the output dtype.
+// With the second level ("HQQ tutorial" (devpress.csdn.net) §3.3, quant_scale/quant_zero),
+// scale_g (zero_g) is first rebuilt in fp32 as (code - zero2)*step2 of its run.
+//
+// Layout on B200: HBM-bound (about 2.5 bytes per weight at 4 bits). A thread writes chunks of
+// 8 consecutive outputs with one 16-byte streaming store each (two for fp32), so a warp stores
+// 512 contiguous bytes per instruction; for axis=1 the 8 codes come from one 1..8-byte load
+// (or two 32-bit words for 3 bits) with one scale/zero pair. Codes become floats through the
+// 2^23 mantissa trick and group indices through shifts, keeping the slow conversion/XU pipe
+// and 64-bit division out of the per-element work.
+#include "hqq_device.cuh"
+#include "hqq_kernels.h"
+
+namespace hqqk {
+
+constexpr int kDBlock = 256;
+
+struct DArgs {
+  const uint8_t* packed;
+  const void* scale;
+  const void* zero;
+  const float* scale_mm;
+  const float* zero_mm;
+  int meta_group_size, meta_dtype;
+  int64_t rows, cols, n;  // n = rows*cols
+  int group_size, log2_group;
+  void* out;
+};
+
+// Small non-negative integer (< 2^23) to fp32 without a conversion instruction: OR it into
+// the mantissa of 2^23 and subtract 2^23 (exact; stays on the FMA/ALU pipes).
+__device__ __forceinline__ float u2f_small(uint32_t q) {
+  return __fsub_rn(__uint_as_float(q | 0x4B000000u), 8388608.0f);
+}
+
+__device__ __forceinline__ float meta_value(const void* p, const float* mm, int mdt, int mgs,
+                                            int64_t g) {
+  if (mm) {
+    const int64_t run = g / mgs;
+    const float q = u2f_small(reinterpret_cast<const uint8_t*>(p)[g]);
+    return __fmul_rn(__fsub_rn(q, mm[2 * run + 1]), mm[2 * run]);
+  }
+  return load_meta(p, mdt, g);
+}
+
+// Code with stream index k (layout of the header).
+template <int NB>
+__device__ __forceinline__ uint32_t code_at(const uint8_t* packed, int64_t k) {
+  if constexpr (NB == 3) {
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(packed) + k / 10);
+    return (w >> (3 * (int)(k % 10))) & 7u;
+  } else {
+    constexpr int PER = 8 / NB;
+    return (__ldg(packed + k / PER) >> ((int)(k % PER) * NB)) & ((1u << NB) - 1u);
+  }
+}
+
+template <int OUT_DT>
+__device__ __forceinline__ void store8(void* out, int64_t k0, const float (&v)[8]) {
+  if constexpr (OUT_DT == kF32) {
+    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + k0);
+    __stcs(dst, make_float4(v[0], v[1], v[2], v[3]));
+    __stcs(dst + 1, make_float4(v[4], v[5], v[6], v[7]));
+  } else {
+    uint4 u;
+    u.x = pack2_16<OUT_DT>(v[0], v[1]);
+    u.y = pack2_16<OUT_DT>(v[2], v[3]);
+    u.z = pack2_16<OUT_DT>(v[4], v[5]);
+    u.w = pack2_16<OUT_DT>(v[6], v[7]);
+    __stcs(reinterpret_cast<uint4*>(reinterpret_cast<unsigned short*>(out) + k0), u);
+  }
+}
+
+template <int OUT_DT>
+__device__ __forceinline__ void store1(void* out, int64_t k, float v) {
+  store_meta(out, OUT_DT, k, v);
+}
+
+// Raw bits of codes k0..k0+7 (k0 a multiple of 8): one 8..64-bit load for 8/4/2/1 bits;
+// for 3 bits the (up to) two 32-bit words they occupy, with the slot of code k0 in `off`.
+template <int NB>
+__device__ __forceinline__ uint64_t codes8_raw(const uint8_t* packed, int64_t k0, int64_t n_codes,
+                                               int& off) {
+  if constexpr (NB == 3) {
+    const uint32_t* wp = reinterpret_cast<const uint32_t*>(packed);
+    const int64_t w0 = k0 / 10;
+    off = (int)(k0 - w0 * 10);
+    const int64_t last = (k0 + 7 < n_codes ? k0 + 7 : n_codes - 1) / 10;
+    const uint32_t lo = __ldg(wp + w0);
+    const uint32_t hi = last > w0 ? __ldg(wp + w0 + 1) : 0u;
+    return (uint64_t)lo | ((uint64_t)hi << 32);
+  } else {
+    off = 0;
+    const uint8_t* src = packed + k0 * NB / 8;
+    if constexpr (NB == 8) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
+      return (uint64_t)v.x | ((uint64_t)v.y << 32);
+    } else if constexpr (NB == 4) {
+      return __ldg(reinterpret_cast<const uint32_t*>(src));
+    } else if constexpr (NB == 2) {
+      return __ldg(reinterpret_cast<const unsigned short*>(src));
+    } else {
+      return __ldg(src);
+    }
+  }
+}
+
+template <int NB>
+__device__ __forceinline__ uint32_t code_in(uint64_t raw, int off, int i) {
+  if constexpr (NB == 3) {
+    const int slot = off + i;  // 0..16: slots 10.. live in the second word
+    const uint32_t w = slot < 10 ? (uint32_t)raw : (uint32_t)(raw >> 32);
+    return (w >> (3 * (slot < 10 ? slot : slot - 10))) & 7u;
+  } else {
+    return (uint32_t)(raw >> (i * NB)) & ((1u << NB) - 1u);
+  }
+}
+
+// axis=1: 8 consecutive elements share one group and have consecutive codes. Grid-stride
+// over chunks of 8 elements at full occupancy; each pass a thread loads kDChunks chunks
+// (kDBlock chunks apart, so a warp's accesses of one chunk index are contiguous) before it
+// computes and stores any, keeping that many loads in flight.
+constexpr int kDChunks = 4;
+
+template <int NB, int OUT_DT>
+__global__ void __launch_bounds__(kDBlock, 6) dequant_axis1_kernel(const DArgs a) {
+  const int64_t n_chunks = a.n >> 3;
+  const int64_t pass = (int64_t)gridDim.x * kDBlock * kDChunks;
+  for (int64_t c0 = (int64_t)blockIdx.x * kDBlock * kDChunks + threadIdx.x; c0 < n_chunks;
+       c0 += pass) {
+    uint64_t raw[kDChunks];
+    int off[kDChunks];
+    float sc[kDChunks], zr[kDChunks];
+#pragma unroll
+    for (int i = 0; i < kDChunks; ++i) {
+      const int64_t c = c0 + (int64_t)i * kDBlock;
+      if (c < n_chunks) {
+        raw[i] = codes8_raw<NB>(a.packed, c << 3, a.n, off[i]);
+        const int64_t g = (c << 3) >> a.log2_group;
+        sc[i] = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g);
+        zr[i] = meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kDChunks; ++i) {
+      const int64_t c = c0 + (int64_t)i * kDBlock;
+      if (c < n_chunks) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          v[j] = __fmul_rn(__fsub_rn(u2f_small(code_in<NB>(raw[i], off[i], j)), zr[i]), sc[i]);
+        store8<OUT_DT>(a.out, c << 3, v);  // n and G are multiples of 8 on this path
+      }
+    }
+  }
+}
+
+// axis=0 (groups run down columns): element (r, c) is code j = r % G of group
+// g = (r / G)*cols + c. Rows with cols % 8 == 0 take 8 columns per thread.
+template <int NB, int OUT_DT>
+__global__ void __launch_bounds__(kDBlock) dequant_axis0_kernel(const DArgs a) {
+  const int64_t k0 = ((int64_t)blockIdx.x * kDBlock + threadIdx.x) * 8;
+  if (k0 >= a.n) return;
+  const int G = a.group_size;
+  if ((a.cols & 7) == 0) {
+    const int64_t r = k0 / a.cols, c0 = k0 - r * a.cols;
+    const int64_t rb = r >> a.log2_group;
+    const int j = (int)(r - (rb << a.log2_group));
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t g = rb * a.cols + c0 + i;
+      const float sc = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g);
+      const float zr = meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g);
+      const float q = u2f_small(code_at<NB>(a.packed, (g << a.log2_group) + j));
+      v[i] = __fmul_rn(__fsub_rn(q, zr), sc);
+    }
+    store8<OUT_DT>(a.out, k0, v);
+    return;
+  }
+  const int64_t kend = k0 + 8 < a.n ? k0 + 8 : a.n;
+  for (int64_t k = k0; k < kend; ++k) {
+    const int64_t r = k / a.cols, c = k - r * a.cols;
+    const int64_t rb = r / G;
+    const int j = (int)(r - rb * G);
+    const int64_t g = rb * a.cols + c;
+    const float sc = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g);
+    const float zr = meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g);
+    const float q = u2f_small(code_at<NB>(a.packed, g * G + j));
+    store1<OUT_DT>(a.out, k, __fmul_rn(__fsub_rn(q, zr), sc));
+  }
+}
+
+// SMs x resident blocks per SM of `kernel` on the current device (host-side query).
+template <typename K>
+static cudaError_t resident_blocks(K kernel, int* out) {
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kDBlock, 0);
+  *out = sms * (per_sm > 0 ? per_sm : 1);
+  return e;
+}
+
+template <int NB, int OUT_DT>
+static cudaError_t launch_nb_dt(const DArgs& a, int axis, cudaStream_t st) {
+  const int64_t threads = (a.n + 7) / 8;
+  const int64_t blocks = (threads + kDBlock - 1) / kDBlock;
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  if (axis == 1) {
+    int resident = 0;
+    const cudaError_t e = resident_blocks(dequant_axis1_kernel<NB, OUT_DT>, &resident);
+    if (e != cudaSuccess) return e;
+    int64_t b1 = (threads + (int64_t)kDBlock * kDChunks - 1) / ((int64_t)kDBlock * kDChunks);
+    if (b1 > resident) b1 = resident;
+    dequant_axis1_kernel<NB, OUT_DT><<<(unsigned)b1, kDBlock, 0, st>>>(a);
+  } else {
+    dequant_axis0_kernel<NB, OUT_DT><<<(unsigned)blocks, kDBlock, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+template <int OUT_DT>
+static cudaError_t launch_dt(const DArgs& a, int nbits, int axis, cudaStream_t st) {
+  switch (nbits) {
+    case 1: return launch_nb_dt<1, OUT_DT>(a, axis, st);
+    case 2: return launch_nb_dt<2, OUT_DT>(a, axis, st);
+    case 3: return launch_nb_dt<3, OUT_DT>(a, axis, st);
+    case 4: return launch_nb_dt<4, OUT_DT>(a, axis, st);
+    default: return launch_nb_dt<8, OUT_DT>(a, axis, st);
+  }
+}
+
+cudaError_t launch_dequantize(const DequantJob& j, cudaStream_t st) {
+  DArgs a;
+  a.packed = j.packed;
+  a.scale = j.scale;
+  a.zero = j.zero;
+  a.scale_mm = j.scale_mm;
+  a.zero_mm = j.zero_mm;
+  a.meta_group_size = j.meta_group_size > 0 ? j.meta_group_size : 1;
+  a.meta_dtype = j.meta_dtype;
+  a.rows = j.rows;
+  a.cols = j.cols;
+  a.n = j.rows * j.cols;
+  a.group_size = j.group_size;
+  a.log2_group = 0;
+  while ((1 << a.log2_group) < j.group_size) ++a.log2_group;
+  a.out = j.out;
+  switch (j.out_dtype) {
+    case kF16: return launch_dt<kF16>(a, j.nbits, j.axis, st);
+    case kBF16: return launch_dt<kBF16>(a, j.nbits, j.axis, st);
+    default: return launch_dt<kF32>(a, j.nbits, j.axis, st);
+  }
+}
+
+// ------------------------------------------------------------------ second level
+
+// One warp per run of `group` values: min/max, step2/zero2, 8-bit codes
+// ("HQQ tutorial" (devpress.csdn.net) §3.3; round-to-nearest only, no solver).
+__global__ void __launch_bounds__(256) quantize_meta_kernel(const void* meta, int dt, int64_t n,
+                                                            int group, uint8_t* q, float* mm) {
+  const int64_t run = ((int64_t)blockIdx.x * 256 + threadIdx.x) / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t runs = (n + group - 1) / group;
+  if (run >= runs) return;
+  const int64_t b = run * group;
+  const int64_t e = b + group < n ? b + group : n;
+  float mn = __int_as_float(0x7f800000), mx = -mn;
+  for (int64_t k = b + lane; k < e; k += 32) {
+    const float v = load_meta(meta, dt, k);
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  float s2 = 1.0f, st2 = 1.0f;
+  if (mx > mn) {
+    const float range = __fsub_rn(mx, mn);
+    s2 = __fdiv_rn(255.0f, range);
+    st2 = __fdiv_rn(range, 255.0f);
+  }
+  const float z2 = __fmul_rn(-mn, s2);
+  for (int64_t k = b + lane; k < e; k += 32) {
+    const float v = __fadd_rn(__fmul_rn(load_meta(meta, dt, k), s2), z2);
+    q[k] = (uint8_t)(__float_as_uint(__fadd_rn(fminf(fmaxf(v, 0.0f), 255.0f), kRoundMagic)) -
+                     0x4B400000u);
+  }
+  if (lane == 0) {
+    mm[2 * run] = st2;
+    mm[2 * run + 1] = z2;
+  }
+}
+
+__global__ void __launch_bounds__(256) dequantize_meta_kernel(const uint8_t* q, const float* mm,
+                                                              int64_t n, int group, float* out) {
+  const int64_t k = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (k >= n) return;
+  const int64_t run = k / group;
+  out[k] = __fmul_rn(__fsub_rn(u2f_small(q[k]), mm[2 * run + 1]), mm[2 * run]);
+}
+
+cudaError_t launch_quantize_meta(const void* meta, int dtype, int64_t n, int group, uint8_t* q,
+                                 float* mm, cudaStream_t st) {
+  const int64_t runs = (n + group - 1) / group;
+  const int64_t blocks = (runs * 32 + 255) / 256;
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  quantize_meta_kernel<<<(unsigned)blocks, 256, 0, st>>>(meta, dtype, n, group, q, mm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize_meta(const uint8_t* q, const float* mm, int64_t n, int group,
+                                   float* out, cudaStream_t st) {
+  const int64_t blocks = (n + 255) / 256;
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  dequantize_meta_kernel<<<(unsigned)blocks, 256, 0, st>>>(q, mm, n, group, out);
+  return cudaGetLastError();
+}
+
+}  // namespace hqqk

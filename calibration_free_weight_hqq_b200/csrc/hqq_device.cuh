@@ -1,0 +1,99 @@
+// hqq_device.cuh - device helpers shared by the quantize, dequantize and meta kernels of
+// the B200 (sm_100a) HQQ library: dtype conversion, MUFU wrappers, rounding, packing.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hqq_kernels.h"
+
+namespace hqqk {
+
+// 1.5 * 2^23: adding then subtracting it rounds an fp32 value |v| < 2^22 to the nearest
+// integer, ties to even (the sum lands in [2^23, 2^24) where the spacing is 1). Both adds
+// run on the FMA pipe, unlike a separate round instruction.
+constexpr float kRoundMagic = 12582912.0f;
+
+__device__ __forceinline__ float rint_magic(float v) {
+  return __fsub_rn(__fadd_rn(v, kRoundMagic), kRoundMagic);
+}
+
+// MUFU base-2 logarithm / exponential (documented PTX approximations, ftz).
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Exact fp32 -> fp64 widening built from the bit fields on the integer pipes (no conversion
+// instruction, which would share the SFU pipe with lg2/ex2). Zero and subnormal inputs, which
+// need renormalisation, take the conversion instruction.
+__device__ __forceinline__ double f32_to_f64_exact(float x) {
+  const uint32_t b = __float_as_uint(x);
+  const uint32_t e = (b >> 23) & 0xffu;
+  if (e == 0u || e == 0xffu) return (double)x;
+  const uint32_t hi = (b & 0x80000000u) | ((e + 896u) << 20) | ((b >> 3) & 0x000fffffu);
+  const uint32_t lo = b << 29;
+  return __hiloint2double((int)hi, (int)lo);
+}
+
+// A non-negative integer below 2^23 held exactly in an fp32, widened to fp64 without a
+// conversion instruction (2^52 + i built from bits, minus 2^52; both exact).
+__device__ __forceinline__ double small_int_f32_to_f64(float x) {
+  const uint32_t i = __float_as_uint(__fadd_rn(x, 8388608.0f)) - 0x4B000000u;
+  return __dsub_rn(__hiloint2double(0x43300000, (int)i), 4503599627370496.0);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
+__device__ __forceinline__ float f16_bits_to_f32(uint32_t h) {
+  return __half2float(__ushort_as_half((unsigned short)h));
+}
+
+// Load one element of dtype DT at index i as fp32 (exact upcast).
+template <int DT>
+__device__ __forceinline__ float load_elem(const void* p, int64_t i) {
+  if constexpr (DT == kF32) {
+    return __ldg(reinterpret_cast<const float*>(p) + i);
+  } else {
+    unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(p) + i);
+    return DT == kBF16 ? bf16_bits_to_f32(h) : f16_bits_to_f32(h);
+  }
+}
+
+__device__ __forceinline__ float load_meta(const void* p, int dt, int64_t i) {
+  if (dt == kF32) return reinterpret_cast<const float*>(p)[i];
+  unsigned short h = reinterpret_cast<const unsigned short*>(p)[i];
+  return dt == kBF16 ? bf16_bits_to_f32(h) : f16_bits_to_f32(h);
+}
+
+// Store an fp32 value rounded once (nearest even) to dtype dt.
+__device__ __forceinline__ void store_meta(void* p, int dt, int64_t i, float v) {
+  if (dt == kF32) {
+    reinterpret_cast<float*>(p)[i] = v;
+  } else if (dt == kBF16) {
+    reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  } else {
+    reinterpret_cast<__half*>(p)[i] = __float2half_rn(v);
+  }
+}
+
+// Round two fp32 values to 16-bit storage and pack them (low half = a).
+template <int DT>
+__device__ __forceinline__ uint32_t pack2_16(float a, float b) {
+  if constexpr (DT == kBF16) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+}  // namespace hqqk

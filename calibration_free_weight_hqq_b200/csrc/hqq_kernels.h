@@ -1,0 +1,48 @@
+// hqq_kernels.h - host-side launch interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hqqk {
+
+// Element types; the values equal the public hqq_dtype enumerators.
+enum Dt : int { kF16 = 0, kBF16 = 1, kF32 = 2, kU8 = 3 };
+
+// One matrix of the quantize path.
+struct QuantJob {
+  const void* W;     // device, row-major [rows, cols]
+  int64_t rows, cols, n_groups;
+  int w_dtype;       // Dt
+  int nbits, group_size, axis, iters;
+  float p, beta0, kappa;
+  uint8_t* packed;   // device, packed code stream
+  void* scale;       // device, n_groups values of scale_dtype
+  void* zero;        // device, n_groups values of zero_dtype
+  int scale_dtype;   // Dt (kF32 when the second level follows)
+  int zero_dtype;
+};
+
+// One matrix of the dequantize path.
+struct DequantJob {
+  const uint8_t* packed;
+  const void* scale;  // meta_dtype values, or uint8 codes when scale_mm != nullptr
+  const void* zero;   // meta_dtype values, or uint8 codes when zero_mm != nullptr
+  const float* scale_mm;  // second-level (step2, zero2) pairs or nullptr
+  const float* zero_mm;
+  int meta_group_size;
+  int meta_dtype;
+  int64_t rows, cols, n_groups;
+  int nbits, group_size, axis;
+  int out_dtype;
+  void* out;
+};
+
+cudaError_t launch_quantize(const QuantJob& job, cudaStream_t stream);
+cudaError_t launch_dequantize(const DequantJob& job, cudaStream_t stream);
+cudaError_t launch_quantize_meta(const void* meta, int dtype, int64_t n, int group, uint8_t* q,
+                                 float* mm, cudaStream_t stream);
+cudaError_t launch_dequantize_meta(const uint8_t* q, const float* mm, int64_t n, int group,
+                                   float* out, cudaStream_t stream);
+
+}  // namespace hqqk

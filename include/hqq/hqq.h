@@ -24,8 +24,10 @@
  *   Pointers   Arguments documented "device" must be device (or managed) memory on the
  *              current device. Host pointers there are undefined behaviour.
  *   Errors     Argument errors are returned synchronously before any launch, and nothing
- *              is written. A failed launch returns HQQ_ERR_CUDA (the CUDA error string is
- *              available from hqq_last_cuda_error()). Nothing throws across this ABI.
+ *              is written. When there is nothing to do (rows*cols == 0, n == 0) a call with
+ *              otherwise valid arguments returns HQQ_OK at once; its pointers may be NULL.
+ *              A failed launch returns HQQ_ERR_CUDA (the CUDA error string is available
+ *              from hqq_last_cuda_error()). Nothing throws across this ABI.
  *   Threads    All entry points are re-entrant. hqq_last_cuda_error() is thread-local.
  *
  * Packed code layout (fixed here; the pages fix none)

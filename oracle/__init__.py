@@ -55,6 +55,8 @@ def _load():
             lib.hqq_oracle_quantize_group.argtypes = [P, i32, i32, i32, f32, f32, f32, P, P, P, P,
                                                       P]
             lib.hqq_oracle_quantize_group.restype = f32
+            lib.hqq_oracle_codes_at_zero.argtypes = [P, i32, i32, f32, P]
+            lib.hqq_oracle_codes_at_zero.restype = None
             lib.hqq_oracle_shrink.argtypes = [f32, f32, f32]
             lib.hqq_oracle_shrink.restype = f32
             lib.hqq_oracle_packed_bytes.argtypes = [i64, i32]
@@ -132,6 +134,14 @@ def quantize_group(w, nbits: int, iters: int, p: float, beta0: float, kappa: flo
                                          _ptr(s), _ptr(z), _ptr(zt), _ptr(et))
     return dict(codes=codes, scale=np.float32(s[0]), zero=np.float32(z[0]),
                 best_err=np.float32(best), z_trace=zt, e_trace=et)
+
+
+def codes_at_zero(w, nbits: int, zero: float) -> np.ndarray:
+    """Final-code step alone for one group at a given zero."""
+    w = _f32(w).ravel()
+    out = np.zeros(w.size, np.uint8)
+    _load().hqq_oracle_codes_at_zero(_ptr(w), w.size, nbits, float(zero), _ptr(out))
+    return out
 
 
 def shrink(r: float, beta: float, p: float) -> np.float32:

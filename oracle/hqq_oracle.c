@@ -170,6 +170,25 @@ float hqq_oracle_quantize_group(const float* w, int G, int nbits, int iters, flo
   return best_e;
 }
 
+/* Step 4 alone for a given zero: the codes clamp(rint(w_j*s + zero), 0, qmax) of one
+ * group with its min/max scale s (used to check a candidate zero chosen elsewhere). */
+void hqq_oracle_codes_at_zero(const float* w, int G, int nbits, float zero, uint8_t* codes) {
+  const float qmax = (float)((1 << nbits) - 1);
+  float mn = w[0], mx = w[0];
+  for (int j = 1; j < G; ++j) {
+    if (w[j] < mn) mn = w[j];
+    if (w[j] > mx) mx = w[j];
+  }
+  float s = 1.0f;
+  if (mx > mn) s = qmax / (mx - mn);
+  for (int j = 0; j < G; ++j) {
+    float q = rintf(w[j] * s + zero);
+    q = fmaxf(q, 0.0f);
+    q = fminf(q, qmax);
+    codes[j] = (uint8_t)q;
+  }
+}
+
 /* Gather group g of a row-major [rows, cols] matrix ([guide 2.2] axis). */
 static void gather_group(const float* W, int64_t rows, int64_t cols, int G, int axis, int64_t g,
                          float* w) {

@@ -1,0 +1,130 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every function that
+include/hqq/hqq.h declares, its size helpers agree with the layout, and argument errors are
+reported synchronously before any CUDA call (fake non-null pointers are never dereferenced
+because every call here fails validation or has nothing to do)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+import torch
+
+import calibration_free_weight_hqq_b200 as hqq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hqq", "hqq.h")
+
+OK, INVALID, UNSUPPORTED, SHAPE, ALIGN, CUDA, WORKSPACE = range(7)
+FAKE = 0x100000  # 16-byte aligned, never dereferenced
+FAKE_ODD = 0x100002
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hqq_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    return hqq.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert "hqq_quantize" in names and "hqq_dequantize" in names and len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.hqq_abi_version() == 1
+
+
+def test_size_helpers_match_layout(L):
+    import oracle
+    for nbits in (1, 2, 3, 4, 8):
+        for rows, cols in ((0, 0), (1, 64), (37, 128), (4096, 1024)):
+            n = rows * cols
+            assert hqq.hqq_packed_bytes(rows, cols, nbits) == oracle.packed_bytes(n, nbits)
+    assert hqq.hqq_packed_bytes(4096, 1024, 5) == 0
+    assert hqq.hqq_num_groups(4096, 1024, 64, 1) == 65536
+    assert hqq.hqq_num_groups(4096, 1024, 64, 0) == 65536
+    assert hqq.hqq_num_groups(100, 1024, 64, 0) == -1
+    assert hqq.hqq_num_groups(100, 1000, 64, 1) == -1
+    assert hqq.hqq_num_groups(64, 64, 48, 1) == -1
+    assert hqq.hqq_num_meta_groups(300, 128) == 3
+    p = hqq.make_params(nbits=3, group_size=64, quant_scale=True, quant_zero=True)
+    ng = 28672 * 8192 // 64
+    assert hqq.hqq_workspace_bytes(28672, 8192, p) == 2 * math.ceil(ng * 4 / 256) * 256
+    p0 = hqq.make_params()
+    assert hqq.hqq_workspace_bytes(28672, 8192, p0) == 0
+
+
+def test_status_strings(L):
+    for code, name in enumerate(["HQQ_OK", "HQQ_ERR_INVALID_ARG", "HQQ_ERR_UNSUPPORTED",
+                                 "HQQ_ERR_SHAPE", "HQQ_ERR_ALIGNMENT", "HQQ_ERR_CUDA",
+                                 "HQQ_ERR_WORKSPACE"]):
+        assert L.hqq_status_string(code).decode() == name
+
+
+def q(L, **kw):
+    a = dict(W=FAKE, dtype=1, rows=64, cols=128, nbits=4, G=64, axis=1, iters=20, p=0.7,
+             beta0=10.0, kappa=1.01, packed=FAKE, scale=FAKE, zero=FAKE)
+    a.update(kw)
+    return L.hqq_quantize(a["W"], a["dtype"], a["rows"], a["cols"], a["nbits"], a["G"],
+                          a["axis"], a["iters"], a["p"], a["beta0"], a["kappa"], a["packed"],
+                          a["scale"], a["zero"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(nbits=5), UNSUPPORTED), (dict(nbits=0), UNSUPPORTED), (dict(G=48), UNSUPPORTED),
+    (dict(G=512), UNSUPPORTED), (dict(axis=2), UNSUPPORTED), (dict(dtype=3), UNSUPPORTED),
+    (dict(cols=100), SHAPE), (dict(axis=0, rows=100), SHAPE), (dict(rows=-1), INVALID),
+    (dict(iters=-1), INVALID), (dict(iters=100000), INVALID), (dict(p=0.0), INVALID),
+    (dict(p=1.5), INVALID), (dict(p=float("nan")), INVALID), (dict(beta0=0.0), INVALID),
+    (dict(beta0=float("inf")), INVALID), (dict(kappa=0.5), INVALID), (dict(W=0), INVALID),
+    (dict(packed=0), INVALID), (dict(scale=0), INVALID), (dict(W=FAKE_ODD), ALIGN),
+    (dict(packed=FAKE + 8), ALIGN), (dict(scale=FAKE + 1), ALIGN),
+    (dict(rows=1 << 30, cols=1 << 30), SHAPE),
+])
+def test_quantize_rejects_bad_arguments(L, kw, status):
+    assert q(L, **kw) == status
+
+
+def test_empty_matrix_is_a_no_op(L):
+    assert q(L, rows=0) == OK
+    assert q(L, cols=0) == OK
+
+
+def test_quantize_ex_workspace_and_meta_checks(L):
+    p = hqq.make_params(quant_scale=True, quant_zero=True)
+    call = lambda **kw: L.hqq_quantize_ex(kw.get("W", FAKE), 64, 128, ctypes.byref(p), FAKE,
+                                          FAKE, FAKE, kw.get("smm", FAKE), kw.get("zmm", FAKE),
+                                          kw.get("ws", FAKE), kw.get("wsb", 0), None)
+    assert call() == WORKSPACE
+    assert call(ws=None, wsb=1 << 20) == WORKSPACE
+    assert call(smm=None, wsb=1 << 20) == INVALID
+    assert call(ws=FAKE + 4, wsb=1 << 20) == ALIGN
+    bad = hqq.make_params(quant_scale=True, meta_group_size=4)
+    assert L.hqq_quantize_ex(FAKE, 64, 128, ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE,
+                             FAKE, 1 << 20, None) == UNSUPPORTED
+    assert L.hqq_quantize_ex(FAKE, 64, 128, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0,
+                             None) == INVALID
+
+
+def test_dequantize_rejects_bad_arguments(L):
+    d = lambda **kw: L.hqq_dequantize(kw.get("pk", FAKE), FAKE, FAKE, kw.get("mdt", 1),
+                                      kw.get("odt", 1), 64, kw.get("cols", 128),
+                                      kw.get("nbits", 4), 64, 1, kw.get("out", FAKE), None)
+    assert d(nbits=6) == UNSUPPORTED
+    assert d(odt=3) == UNSUPPORTED
+    assert d(cols=96) == SHAPE
+    assert d(out=0) == INVALID
+    assert d(out=FAKE + 2) == ALIGN
+    assert L.hqq_dequantize_meta(FAKE, FAKE, 100, 3, FAKE, None) == UNSUPPORTED
+    assert L.hqq_quantize_meta(FAKE, 1, -1, 128, FAKE, FAKE, None) == INVALID
+
+
+def test_binding_has_no_cpu_path():
+    W = torch.zeros(64, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        hqq.hqq_quantize(W)

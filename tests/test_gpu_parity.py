@@ -1,0 +1,250 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs, element by element, within the tolerances stated in tests/parity.py.
+
+Covers the five shipped workloads (full matrices where the oracle finishes in seconds,
+seeded group samples that always include the ragged tail otherwise), every nbits, group
+size, axis and dtype on small ragged shapes, and the edge cases: empty input, constant
+groups, an active shrinkage, iters = 0, canary bytes past the outputs, stored meta dtypes,
+determinism and a matrix with more than 2^32 elements."""
+import numpy as np
+import pytest
+import torch
+
+import calibration_free_weight_hqq_b200 as hqq
+from calibration_free_weight_hqq_b200 import synthetic, workloads
+import oracle
+from parity import compare, group_view, sample_groups, unpack_groups
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def W_of(m):
+    return workloads.make_weight(m, device=DEV)
+
+
+# ------------------------------------------------------------------ shipped workloads
+
+
+def test_single_fp16_full():
+    """[4096,1024] fp16, 4-bit g64 axis 1: every group compared."""
+    m = workloads.single_fp16().matrices[0]
+    r = compare(W_of(m), 4, 64, 1)
+    print(r)
+    r.check()
+
+
+@pytest.mark.parametrize("i", range(7))
+def test_llama7b_block_4b(i):
+    m = workloads.llama7b_block_4b().matrices[i]
+    r = compare(W_of(m), m.nbits, m.group_size, m.axis, n_sample=40000, seed=i)
+    print(m.name, r)
+    r.check()
+
+
+@pytest.mark.parametrize("i", range(7))
+def test_llama7b_block_2b_axis0(i):
+    m = workloads.llama7b_block_2b_axis0().matrices[i]
+    r = compare(W_of(m), m.nbits, m.group_size, m.axis, n_sample=100000, seed=i)
+    print(m.name, r)
+    r.check()
+
+
+@pytest.mark.parametrize("i", range(2))
+def test_mlp70b_mixed_with_meta(i):
+    m = workloads.mlp70b_mixed().matrices[i]
+    r = compare(W_of(m), m.nbits, m.group_size, m.axis, n_sample=60000, seed=i,
+                quant_meta=True, meta_group=m.meta_group_size)
+    print(m.name, r)
+    r.check()
+
+
+def test_llama7b_model_sampled():
+    """Whole 7B-shaped model: all 224 matrices on the GPU, 512 sampled groups of each."""
+    wl = workloads.llama7b_model_4b()
+    total = None
+    for i, m in enumerate(wl.matrices):
+        r = compare(W_of(m), m.nbits, m.group_size, m.axis, n_sample=512, seed=i)
+        r.check()
+        total = r if total is None else _acc(total, r)
+    print(total)
+
+
+def _acc(a, b):
+    for f in ("n_groups", "n_codes", "scale_exact", "zero_exact", "zero_diverged", "code_diff"):
+        setattr(a, f, getattr(a, f) + getattr(b, f))
+    return a
+
+
+# ------------------------------------------------------------------ coverage grid
+
+
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("G", [8, 16, 32, 64, 128, 256])
+@pytest.mark.parametrize("axis", [0, 1])
+def test_grid_ragged(nbits, G, axis):
+    """Ragged shapes: >= 10^4 groups (so that the 0.01 % rate admits one event), group
+    count not a multiple of the 160-group block."""
+    shape = (837, 12 * G) if axis == 1 else (11 * G, 1000)
+    W = synthetic.weight(*shape, seed=1000 + nbits * 10 + G + axis, dtype=torch.bfloat16,
+                         outlier_rate=0.01, device=DEV)
+    compare(W, nbits, G, axis).check()
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("axis", [0, 1])
+def test_input_dtypes(dtype, axis):
+    W = synthetic.weight(1024, 1024, seed=7, dtype=dtype, outlier_rate=0.002, device=DEV)
+    compare(W, 4, 64, axis).check()
+
+
+@pytest.mark.parametrize("p,beta0,kappa,iters", [(1.0, 10.0, 1.01, 20), (0.5, 3.0, 1.05, 20),
+                                                 (0.7, 10.0, 1.01, 0), (0.7, 10.0, 1.01, 1),
+                                                 (0.7, 10.0, 1.01, 57)])
+def test_solver_constants(p, beta0, kappa, iters):
+    W = synthetic.weight(1024, 1024, seed=11, dtype=torch.bfloat16, device=DEV)
+    r = compare(W, 4, 64, 1, iters=iters, p=p, beta0=beta0, kappa=kappa)
+    r.check()
+    if iters == 0:  # pure RTN: everything bit-exact
+        assert r.zero_exact == r.n_groups and r.code_diff == 0
+
+
+def test_active_shrinkage():
+    """Weights with sigma ~ 1 at 2 bits and beta0 = 1: residuals exceed the shrinkage
+    cut-off, so the exact per-element path runs on most groups and iterations."""
+    W = synthetic.weight(512, 1024, seed=12, dtype=torch.float32, sigma_layer=1.0, device=DEV)
+    r = compare(W, 2, 16, 1, beta0=1.0, kappa=1.1)
+    print(r)
+    r.check()
+    W = synthetic.weight(512, 1024, seed=13, dtype=torch.bfloat16, outlier_rate=0.02,
+                         device=DEV)
+    r = compare(W, 1, 32, 1)
+    print(r)
+    r.check()
+
+
+def test_constant_groups():
+    W = synthetic.weight(1024, 1024, seed=14, dtype=torch.bfloat16, device=DEV)
+    W[5] = 0.25
+    W[9, :64] = -1.0
+    W[17] = 0
+    r = compare(W, 4, 64, 1)
+    r.check()
+    pk, s, z = hqq.hqq_quantize(W, 4, 64, 1)
+    assert torch.all(s[5] == 1) and torch.all(z[5] == -0.25) and torch.all(z[17] == 0)
+    assert s[9, 0] == 1 and z[9, 0] == 1.0
+    codes = oracle.unpack(pk.cpu().numpy(), W.numel(), 4).reshape(1024, 1024)
+    assert np.all(codes[5] == 0) and np.all(codes[17] == 0) and np.all(codes[9, :64] == 0)
+
+
+# ------------------------------------------------------------------ edge cases
+
+
+def test_empty_inputs_write_nothing():
+    W = torch.empty(0, 1024, dtype=torch.bfloat16, device=DEV)
+    pk = torch.full((16,), 0xAB, dtype=torch.uint8, device=DEV)
+    s = torch.full((4,), 7.0, dtype=torch.bfloat16, device=DEV)
+    hqq.hqq_quantize(W, Wq_packed=pk, scale=s, zero=s)
+    torch.cuda.synchronize()
+    assert torch.all(pk == 0xAB) and torch.all(s == 7.0)
+
+
+@pytest.mark.parametrize("nbits,G", [(3, 64), (4, 64), (2, 16), (1, 32), (8, 8)])
+def test_no_write_past_outputs(nbits, G):
+    rows, cols = 3, G * 5
+    W = synthetic.weight(rows, cols, seed=15, dtype=torch.bfloat16, device=DEV)
+    nb = hqq.hqq_packed_bytes(rows, cols, nbits)
+    buf = torch.full((nb + 64,), 0xCD, dtype=torch.uint8, device=DEV)
+    ng = rows * cols // G
+    sbuf = torch.full((ng + 8,), 3.0, dtype=torch.bfloat16, device=DEV)
+    zbuf = torch.full((ng + 8,), 3.0, dtype=torch.bfloat16, device=DEV)
+    hqq.hqq_quantize(W, nbits, G, 1, Wq_packed=buf[:nb], scale=sbuf[:ng], zero=zbuf[:ng])
+    torch.cuda.synchronize()
+    assert torch.all(buf[nb:] == 0xCD)
+    assert torch.all(sbuf[ng:] == 3.0) and torch.all(zbuf[ng:] == 3.0)
+    if nbits == 3:  # 15 groups * 64 codes = 960 codes = 96 words exactly; bits 30-31 zero
+        words = buf[:nb].view(torch.int32).cpu().numpy().view(np.uint32)
+        assert np.all(words >> 30 == 0)
+
+
+def test_three_bit_tail_word_is_zero_padded():
+    W = synthetic.weight(3, 64, seed=16, dtype=torch.bfloat16, device=DEV)  # 192 codes
+    pk, s, z = hqq.hqq_quantize(W, 3, 64, 1)
+    words = pk.view(torch.int32).cpu().numpy().view(np.uint32)
+    assert words.size == 20
+    assert words[-1] >> 6 == 0  # only codes 190, 191 live in the last word
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_stored_meta_dtype_is_rounded_once(dtype):
+    """Flat ABI: scale/zero stored in W's dtype = the fp32 values rounded to nearest even."""
+    W = synthetic.weight(256, 1024, seed=17, dtype=dtype, device=DEV)
+    pk, s, z = hqq.hqq_quantize(W, 4, 64, 1)
+    params = hqq.make_params(4, 64, 1, w_dtype=dtype, meta_dtype=torch.float32)
+    ref = hqq.hqq_quantize_ex(W, params)
+    assert torch.equal(ref["Wq_packed"], pk)
+    assert torch.equal(ref["scale"].to(dtype), s) and torch.equal(ref["zero"].to(dtype), z)
+    # and the stored-dtype values against the oracle's fp32 results rounded the same way
+    Wg = W.float().reshape(-1, 64).cpu().numpy()
+    _, os_, oz = oracle.quantize(Wg, 4, 64, 1, 20, 0.7, 10.0, 1.01, nthreads=8)
+    o_s = torch.from_numpy(os_).to(dtype)
+    assert torch.equal(o_s, s.reshape(-1).cpu())
+    o_z = torch.from_numpy(oz).to(dtype)
+    assert (o_z != z.reshape(-1).cpu()).sum().item() <= 1e-4 * oz.size
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float16, torch.bfloat16, torch.float32])
+def test_dequantize_out_dtypes_bit_exact(out_dtype):
+    W = synthetic.weight(128, 512, seed=18, dtype=torch.bfloat16, device=DEV)
+    pk, s, z = hqq.hqq_quantize(W, 4, 64, 1)
+    D = hqq.hqq_dequantize(pk, s, z, 128, 512, 4, 64, 1, out_dtype=out_dtype)
+    codes = oracle.unpack(pk.cpu().numpy(), 128 * 512, 4)
+    ref = oracle.dequantize(codes, s.float().reshape(-1).cpu().numpy(),
+                            z.float().reshape(-1).cpu().numpy(), 128, 512, 64, 1)
+    assert torch.equal(torch.from_numpy(ref).to(out_dtype), D.cpu())
+
+
+def test_quantize_meta_standalone():
+    m = (torch.randn(1000, device=DEV) * 0.01 + 0.03).float()
+    q, mm = hqq.hqq_quantize_meta(m, 128)
+    oq, omm = oracle.quantize_meta(m.cpu().numpy(), 128)
+    assert np.array_equal(q.cpu().numpy(), oq)
+    assert np.array_equal(mm.cpu().numpy().view(np.uint32), omm.view(np.uint32))
+    back = hqq.hqq_dequantize_meta(q, mm, 128)
+    ob = oracle.dequantize_meta(oq, omm, 128)
+    assert np.array_equal(back.cpu().numpy().view(np.uint32), ob.view(np.uint32))
+
+
+def test_deterministic():
+    W = synthetic.weight(1024, 4096, seed=19, dtype=torch.bfloat16, device=DEV)
+    a = hqq.hqq_quantize(W, 4, 64, 1)
+    b = hqq.hqq_quantize(W, 4, 64, 1)
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+
+
+def test_more_than_2_pow_32_elements():
+    """[65536, 65600] bf16 (4.3e9 weights, 8.6 GB): 64-bit indexing end to end; groups near
+    the end of the matrix are compared with the oracle."""
+    rows, cols, G = 65536, 65600, 64
+    W = torch.empty(rows, cols, dtype=torch.bfloat16, device=DEV)
+    step = 2048
+    for r0 in range(0, rows, step):
+        W[r0:r0 + step] = synthetic.weight(step, cols, seed=20 + r0, dtype=torch.bfloat16,
+                                           device=DEV)
+    pk, s, z = hqq.hqq_quantize(W, 4, G, 1)
+    torch.cuda.synchronize()
+    ng = rows * cols // G
+    ids = np.concatenate([np.arange(ng - 3000, ng), np.arange(2 ** 26, 2 ** 26 + 1000),
+                          np.arange(0, 1000)]).astype(np.int64)
+    ids_t = torch.from_numpy(ids).to(DEV)
+    Wg = W.reshape(ng, G)[ids_t].float().cpu().numpy()
+    oc, os_, oz = oracle.quantize(Wg, 4, G, 1, 20, 0.7, 10.0, 1.01, nthreads=8)
+    per = G * 4 // 8
+    pkg = pk.reshape(ng, per)[ids_t].cpu().numpy()
+    gc = oracle.unpack(pkg.ravel(), ids.size * G, 4).reshape(-1, G)
+    assert np.count_nonzero(gc != oc) <= 1e-3 * gc.size
+    assert torch.equal(s.reshape(-1)[ids_t].cpu(), torch.from_numpy(os_).to(torch.bfloat16))
+    del W
+    torch.cuda.empty_cache()
