@@ -19,6 +19,27 @@ namespace hqqk {
 
 constexpr int kDBlock = 256;
 
+// Tuning knobs (compile-time): chunks of 8 elements in flight per thread, streaming
+// (evict-first) output stores, minimum resident blocks per SM.
+#ifndef HQQ_DQ_CHUNKS
+#define HQQ_DQ_CHUNKS 2
+#endif
+#ifndef HQQ_DQ_STCS
+#define HQQ_DQ_STCS 1
+#endif
+#ifndef HQQ_DQ_MINB
+#define HQQ_DQ_MINB 8
+#endif
+
+template <typename T>
+__device__ __forceinline__ void st_out(T* p, const T& v) {
+#if HQQ_DQ_STCS
+  __stcs(p, v);
+#else
+  *p = v;
+#endif
+}
+
 struct DArgs {
   const uint8_t* packed;
   const void* scale;
@@ -63,15 +84,15 @@ template <int OUT_DT>
 __device__ __forceinline__ void store8(void* out, int64_t k0, const float (&v)[8]) {
   if constexpr (OUT_DT == kF32) {
     float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + k0);
-    __stcs(dst, make_float4(v[0], v[1], v[2], v[3]));
-    __stcs(dst + 1, make_float4(v[4], v[5], v[6], v[7]));
+    st_out(dst, make_float4(v[0], v[1], v[2], v[3]));
+    st_out(dst + 1, make_float4(v[4], v[5], v[6], v[7]));
   } else {
     uint4 u;
     u.x = pack2_16<OUT_DT>(v[0], v[1]);
     u.y = pack2_16<OUT_DT>(v[2], v[3]);
     u.z = pack2_16<OUT_DT>(v[4], v[5]);
     u.w = pack2_16<OUT_DT>(v[6], v[7]);
-    __stcs(reinterpret_cast<uint4*>(reinterpret_cast<unsigned short*>(out) + k0), u);
+    st_out(reinterpret_cast<uint4*>(reinterpret_cast<unsigned short*>(out) + k0), u);
   }
 }
 
@@ -124,10 +145,10 @@ __device__ __forceinline__ uint32_t code_in(uint64_t raw, int off, int i) {
 // over chunks of 8 elements at full occupancy; each pass a thread loads kDChunks chunks
 // (kDBlock chunks apart, so a warp's accesses of one chunk index are contiguous) before it
 // computes and stores any, keeping that many loads in flight.
-constexpr int kDChunks = 4;
+constexpr int kDChunks = HQQ_DQ_CHUNKS;
 
 template <int NB, int OUT_DT>
-__global__ void __launch_bounds__(kDBlock, 6) dequant_axis1_kernel(const DArgs a) {
+__global__ void __launch_bounds__(kDBlock, HQQ_DQ_MINB) dequant_axis1_kernel(const DArgs a) {
   const int64_t n_chunks = a.n >> 3;
   const int64_t pass = (int64_t)gridDim.x * kDBlock * kDChunks;
   for (int64_t c0 = (int64_t)blockIdx.x * kDBlock * kDChunks + threadIdx.x; c0 < n_chunks;

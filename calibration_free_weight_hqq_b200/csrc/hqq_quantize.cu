@@ -323,7 +323,7 @@ __device__ __forceinline__ void solve_group(const QArgs& a, int64_t g, int lane,
     // Closed-form zero. Every lane computes it (a masked warp instruction costs the pipe as
     // much as a full one, so one lane computing and broadcasting would only add a shuffle).
     const double num = __dadd_rn(__dsub_rn(small_int_f32_to_f64(sq), S_ws), __dmul_rn(s_d, swe));
-    z = __double2float_rn(num * (1.0 / (double)G));  // G is a power of two: exact
+    z = __double2float_rn(__dmul_rn(num, 1.0 / (double)G));  // G is a power of two: exact
     beta = __fmul_rn(beta, a.kappa);
   }
 
