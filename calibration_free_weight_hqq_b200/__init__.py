@@ -81,10 +81,12 @@ def lib() -> ctypes.CDLL:
                                           P, sz, P]
             L.hqq_dequantize_ex.argtypes = [P, P, P, P, P, i64, i64, ctypes.POINTER(HQQParams),
                                             i32, P, P]
+            L.hqq_quantize_ex_noalloc.argtypes = [P, i64, i64, ctypes.POINTER(HQQParams), P, P,
+                                                  P, P, P, P]
             L.hqq_quantize_meta.argtypes = [P, i32, i64, i32, P, P, P]
             L.hqq_dequantize_meta.argtypes = [P, P, i64, i32, P, P]
             for f in ("hqq_quantize", "hqq_dequantize", "hqq_quantize_ex", "hqq_dequantize_ex",
-                      "hqq_quantize_meta", "hqq_dequantize_meta"):
+                      "hqq_quantize_meta", "hqq_dequantize_meta", "hqq_quantize_ex_noalloc"):
                 getattr(L, f).restype = i32
             L.hqq_packed_bytes.argtypes = [i64, i64, i32, i32, i32]
             L.hqq_packed_bytes.restype = sz
@@ -213,6 +215,37 @@ def hqq_quantize_ex(W: torch.Tensor, params: HQQParams, *, stream=None, workspac
         workspace.data_ptr() if workspace is not None else None,
         workspace.numel() if workspace is not None else 0, _stream(stream))
     _check(st, "hqq_quantize_ex")
+    return out
+
+
+def hqq_quantize_ex_noalloc(W: torch.Tensor, params: HQQParams, *, stream=None):
+    """hqq_quantize_ex whose second-level scratch is the library's fixed device array
+    (HQQ_NOALLOC_SCRATCH_BYTES) instead of a workspace; the outputs are still allocated here
+    (by torch) unless a caller passes its own through the C entry point."""
+    rows, cols = W.shape
+    dev = W.device
+    ng = hqq_num_groups(rows, cols, params.group_size, params.axis)
+    if ng < 0:
+        raise HQQError(3, "hqq_quantize_ex_noalloc")
+    ms = _meta_shape(rows, cols, params.group_size, params.axis)
+    mdt = _DT_TORCH[params.meta_dtype]
+    runs = max(hqq_num_meta_groups(ng, params.meta_group_size), 0)
+    out = {
+        "Wq_packed": torch.empty(hqq_packed_bytes(rows, cols, params.nbits), dtype=torch.uint8,
+                                 device=dev),
+        "scale": torch.empty(ms, dtype=torch.uint8 if params.quant_scale else mdt, device=dev),
+        "zero": torch.empty(ms, dtype=torch.uint8 if params.quant_zero else mdt, device=dev),
+        "scale_mm": torch.empty((runs, 2), dtype=torch.float32, device=dev)
+        if params.quant_scale else None,
+        "zero_mm": torch.empty((runs, 2), dtype=torch.float32, device=dev)
+        if params.quant_zero else None,
+    }
+    st = lib().hqq_quantize_ex_noalloc(
+        _cuda(W, "W"), rows, cols, ctypes.byref(params), _cuda(out["Wq_packed"], "Wq_packed"),
+        _cuda(out["scale"], "scale"), _cuda(out["zero"], "zero"),
+        out["scale_mm"].data_ptr() if out["scale_mm"] is not None else None,
+        out["zero_mm"].data_ptr() if out["zero_mm"] is not None else None, _stream(stream))
+    _check(st, "hqq_quantize_ex_noalloc")
     return out
 
 

@@ -17,7 +17,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 BUILD_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libhqq_b200.so")
-SOURCES = ["hqq_abi.cu", "hqq_quantize.cu", "hqq_dequantize.cu"]
+SOURCES = ["hqq_abi.cu", "hqq_quantize.cu", "hqq_dequantize.cu", "hqq_noalloc.cu"]
 HEADERS = ["hqq_device.cuh", "hqq_kernels.h"]
 PUBLIC_HEADER = os.path.join(ROOT, "include", "hqq", "hqq.h")
 

@@ -169,6 +169,35 @@ hqq_status hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, const hqq_
                            void* Wq_packed, void* scale, void* zero, void* scale_mm, void* zero_mm,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Size of the fixed device scratch that hqq_quantize_ex_noalloc uses in place of a workspace:
+ * 32 MiB, enough for 4,194,304 groups when both quant_scale and quant_zero are set and
+ * 8,388,608 groups when one of them is. */
+#define HQQ_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* hqq_quantize_ex for callers that cannot allocate device memory. (The pages have no
+ * counterpart; this is a deployment convenience of this library.)
+ * Some callers can't call cudaMalloc: a plugin or extension that its host framework hands
+ * only a stream and the tensors, code that runs where every byte of device memory belongs to
+ * another allocator (a caching allocator or a fixed-size pool), or a serving process that
+ * forbids allocation once it has started. The second level needs fp32 scratch for the scale
+ * and zero of every group; this entry point takes it from a fixed array compiled into the
+ * library instead of a caller-supplied workspace, and calls no allocating routine.
+ *   Arguments, outputs and results are those of hqq_quantize_ex without the workspace.
+ *   The array holds HQQ_NOALLOC_SCRATCH_BYTES; a call that needs more
+ *   (hqq_workspace_bytes() > HQQ_NOALLOC_SCRATCH_BYTES) returns HQQ_ERR_WORKSPACE and
+ *   launches nothing. Calls without quant_scale/quant_zero use no scratch.
+ *   Every GPU that loads the array holds it (32 MiB) until the process exits.
+ *   The first call on a device sets up the array's device address for that device (a host
+ *   runtime query, with the device current); make that first call before any stream capture.
+ *   All calls on a device share the one array and it keeps the last call's contents (each
+ *   call writes the parts it reads first, so nothing needs clearing). Calls that overlap on
+ *   the GPU - on different streams, or from different host threads, at the same time on one
+ *   device - race on it: keep such calls ordered, e.g. on one stream. */
+hqq_status hqq_quantize_ex_noalloc(const void* W, int64_t rows, int64_t cols,
+                                   const hqq_params* params, void* Wq_packed, void* scale,
+                                   void* zero, void* scale_mm, void* zero_mm,
+                                   cudaStream_t stream);
+
 /* Inverse of hqq_quantize_ex. When quant_scale (quant_zero) is set, the scale (zero) of each
  * group is first rebuilt in fp32 as (code - zero2)*step2 of its run, and that fp32 value is
  * used directly. W_out as in hqq_dequantize. */
