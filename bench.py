@@ -219,15 +219,27 @@ def run_ours(args, rank, world, dev):
     return res
 
 
+def solver_source_digest() -> str:
+    """sha1 of the solver's sources, to tell whether a recorded capture is still current."""
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("hqq_quantize.cu", "hqq_device.cuh"):
+        with open(os.path.join(HERE, "calibration_free_weight_hqq_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 def _traffic_per_launch(avg_weights):
-    """DRAM bytes of one solver launch, from the committed ncu capture (bytes per weight
-    measured on a [16384,8192] bf16 launch, scaled to the average launch here); None if no
-    capture of the current kernel is recorded."""
+    """DRAM bytes (read + write) of one solver launch, from the committed ncu capture
+    (bytes per weight measured on one [16384, 8192] bf16 launch, scaled to the average launch
+    here). None if no capture is recorded or the solver changed since it was taken."""
     path = os.path.join(HERE, "profiles", "quantize_kernel_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         t = json.load(f)
+    if t.get("solver_source_sha1") != solver_source_digest():
+        return None
     return round(t["dram_bytes_per_weight"] * avg_weights)
 
 
@@ -351,6 +363,70 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def probe_sfu():
+    """Measured lg2/ex2 issue rate per SM per clock (the solver's bound), from the probe
+    kernel in csrc/hqq_probe.cu; clocks sampled meanwhile."""
+    import ctypes
+    L = ctypes.CDLL(os.path.join(HERE, "calibration_free_weight_hqq_b200", "libhqq_probe.so"))
+    L.hqq_probe_sfu.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                ctypes.c_int, ctypes.c_void_p]
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    res = {"probe": "sfu", "sms": sms}
+    with ClockSampler(0) as clk:
+        for op, per, name in ((0, 1, "ex2"), (1, 1, "lg2"), (2, 2, "lg2+ex2")):
+            blocks, threads, iters = sms * 8, 256, 4096
+            out = torch.empty(blocks * threads, device="cuda")
+            st = torch.cuda.current_stream()
+            for _ in range(2):
+                assert L.hqq_probe_sfu(op, out.data_ptr(), blocks, threads, iters, st.cuda_stream) == 0
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            L.hqq_probe_sfu(op, out.data_ptr(), blocks, threads, iters, st.cuda_stream)
+            e1.record(st)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            ops = blocks * threads * iters * 8 * per
+            res[name] = {"ms": round(ms, 3), "ops_per_s": ops / (ms * 1e-3)}
+    c = clk.summary()
+    res["clocks"] = c
+    # The probe runs for milliseconds, shorter than the 200 ms clock sampling, so the rate
+    # is normalised at the maximum SM clock (the clock held under the bench's sustained load).
+    mhz = c.get("sm_max_mhz") or SM_MAX_MHZ
+    res["normalised_at_mhz"] = mhz
+    for name in ("ex2", "lg2", "lg2+ex2"):
+        res[name]["per_clk_per_sm"] = round(res[name]["ops_per_s"] / sms / (mhz * 1e6), 2)
+    return res
+
+
+def single(kind: str, reps: int = 10):
+    """One [16384, 8192] bf16 matrix (134M weights, 268 MB: larger than L2), 4-bit g64:
+    time `reps` solver or dequantize launches after warm-up (the small case the ncu
+    captures in profiles/ use)."""
+    import calibration_free_weight_hqq_b200 as hqq
+    from calibration_free_weight_hqq_b200 import synthetic
+    rows, cols = 16384, 8192
+    W = synthetic.weight(rows, cols, seed=5, dtype=torch.bfloat16, device="cuda")
+    pk, s, z = hqq.hqq_quantize(W, 4, 64, 1)
+    D = torch.empty_like(W)
+    run = (lambda: hqq.hqq_quantize(W, 4, 64, 1, Wq_packed=pk, scale=s, zero=z)) \
+        if kind == "quantize" else \
+        (lambda: hqq.hqq_dequantize(pk, s, z, rows, cols, 4, 64, 1, out=D))
+    for _ in range(2):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    n = rows * cols
+    return {"single": kind, "shape": [rows, cols], "ms": round(ms, 4),
+            "Gweights_per_s": round(n / ms / 1e6, 2),
+            "GB_per_s_algorithmic": round(n * 2.5625 / ms / 1e6, 1)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -360,7 +436,17 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--probe-sfu", action="store_true",
+                    help="measure the lg2/ex2 issue rate behind the roofline peak and exit")
+    ap.add_argument("--single", choices=["quantize", "dequantize"],
+                    help="time one [16384,8192] matrix (the profiling case) and exit")
     args = ap.parse_args()
+    if args.probe_sfu:
+        print(json.dumps(probe_sfu()), flush=True)
+        return
+    if args.single:
+        print(json.dumps(single(args.single)), flush=True)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
