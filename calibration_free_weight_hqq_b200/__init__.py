@@ -49,6 +49,13 @@ class HQQError(RuntimeError):
         super().__init__(f"{where}: {name}" + (f" ({detail})" if detail else ""))
 
 
+class HQQMatrix(ctypes.Structure):
+    """Mirror of the C struct hqq_matrix (one matrix of a batched call)."""
+    _fields_ = [("W", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("Wq_packed", ctypes.c_void_p), ("scale", ctypes.c_void_p),
+                ("zero", ctypes.c_void_p)]
+
+
 class HQQParams(ctypes.Structure):
     """Mirror of the C struct hqq_params."""
     _fields_ = [("nbits", ctypes.c_int), ("group_size", ctypes.c_int), ("axis", ctypes.c_int),
@@ -83,10 +90,15 @@ def lib() -> ctypes.CDLL:
                                             i32, P, P]
             L.hqq_quantize_ex_noalloc.argtypes = [P, i64, i64, ctypes.POINTER(HQQParams), P, P,
                                                   P, P, P, P]
+            L.hqq_quantize_batched.argtypes = [ctypes.POINTER(HQQMatrix), i32,
+                                               ctypes.POINTER(HQQParams), P]
+            L.hqq_dequantize_batched.argtypes = [ctypes.POINTER(HQQMatrix), i32,
+                                                 ctypes.POINTER(HQQParams), i32, P]
             L.hqq_quantize_meta.argtypes = [P, i32, i64, i32, P, P, P]
             L.hqq_dequantize_meta.argtypes = [P, P, i64, i32, P, P]
             for f in ("hqq_quantize", "hqq_dequantize", "hqq_quantize_ex", "hqq_dequantize_ex",
-                      "hqq_quantize_meta", "hqq_dequantize_meta", "hqq_quantize_ex_noalloc"):
+                      "hqq_quantize_meta", "hqq_dequantize_meta", "hqq_quantize_ex_noalloc",
+                      "hqq_quantize_batched", "hqq_dequantize_batched"):
                 getattr(L, f).restype = i32
             L.hqq_packed_bytes.argtypes = [i64, i64, i32, i32, i32]
             L.hqq_packed_bytes.restype = sz
@@ -247,6 +259,57 @@ def hqq_quantize_ex_noalloc(W: torch.Tensor, params: HQQParams, *, stream=None):
         out["zero_mm"].data_ptr() if out["zero_mm"] is not None else None, _stream(stream))
     _check(st, "hqq_quantize_ex_noalloc")
     return out
+
+
+def alloc_outputs(shapes, params: HQQParams, device="cuda"):
+    """(packed, scale, zero) tensors for each (rows, cols) in `shapes`."""
+    mdt = _DT_TORCH[params.meta_dtype]
+    outs = []
+    for rows, cols in shapes:
+        ms = _meta_shape(rows, cols, params.group_size, params.axis)
+        outs.append((torch.empty(hqq_packed_bytes(rows, cols, params.nbits), dtype=torch.uint8,
+                                 device=device),
+                     torch.empty(ms, dtype=mdt, device=device),
+                     torch.empty(ms, dtype=mdt, device=device)))
+    return outs
+
+
+def matrix_batch(Ws, outs):
+    """ctypes array of hqq_matrix descriptors for tensors Ws[i] (inputs of a quantize or
+    outputs of a dequantize) and their (packed, scale, zero) outs[i]; build it once and
+    reuse it across calls to skip the per-call marshalling."""
+    arr = (HQQMatrix * len(Ws))()
+    for i, (W, (pk, sc, zr)) in enumerate(zip(Ws, outs)):
+        arr[i] = HQQMatrix(_cuda(W, "W"), W.shape[0], W.shape[1], _cuda(pk, "Wq_packed"),
+                           _cuda(sc, "scale"), _cuda(zr, "zero"))
+    return arr
+
+
+def hqq_quantize_batched(Ws, params: HQQParams, *, outs=None, batch=None, stream=None):
+    """Quantize a list of 2-D CUDA weights sharing one configuration in as few launches as
+    possible (the whole-model driver). Returns the list of (packed, scale, zero)."""
+    if outs is None:
+        outs = alloc_outputs([tuple(W.shape) for W in Ws], params, Ws[0].device)
+    if batch is None:
+        batch = matrix_batch(Ws, outs)
+    st = lib().hqq_quantize_batched(batch, len(Ws), ctypes.byref(params), _stream(stream))
+    _check(st, "hqq_quantize_batched")
+    return outs
+
+
+def hqq_dequantize_batched(outs, shapes, params: HQQParams, out_dtype=torch.bfloat16, *,
+                           W_out=None, batch=None, stream=None):
+    """Dequantize a list of (packed, scale, zero) of one configuration into new (or given)
+    [rows, cols] tensors of out_dtype."""
+    if W_out is None:
+        W_out = [torch.empty(sh, dtype=out_dtype, device=outs[0][0].device) for sh in shapes]
+    if batch is None:
+        batch = matrix_batch(W_out, outs)
+    st = lib().hqq_dequantize_batched(batch, len(W_out), ctypes.byref(params),
+                                      _TORCH_DT.get(W_out[0].dtype if W_out else out_dtype, -1),
+                                      _stream(stream))
+    _check(st, "hqq_dequantize_batched")
+    return W_out
 
 
 def hqq_dequantize(Wq_packed, scale, zero, rows: int, cols: int, nbits: int = 4,

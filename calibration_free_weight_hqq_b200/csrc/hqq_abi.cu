@@ -5,6 +5,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <vector>
+
 #include "../../include/hqq/hqq.h"
 #include "hqq_kernels.h"
 
@@ -260,6 +262,97 @@ HQQ_EXPORT hqq_status hqq_dequantize_ex(const void* Wq_packed, const void* scale
   return dequantize_impl(Wq_packed, scale, zero, smm, zmm, params->meta_dtype,
                          params->meta_group_size, rows, cols, params->nbits, params->group_size,
                          params->axis, out_dtype, W_out, stream);
+}
+
+// Per-matrix checks shared by the batched calls (shape, pointers, alignment).
+static hqq_status check_matrix(const hqq_matrix& m, const hqq_params& prm, size_t w_align,
+                               int out_dtype) {
+  hqq_status st = check_shape(m.rows, m.cols, prm.nbits, prm.group_size, prm.axis);
+  if (st != HQQ_OK) return st;
+  if (m.rows * m.cols == 0) return HQQ_OK;
+  if (!m.W || !m.Wq_packed || !m.scale || !m.zero) return HQQ_ERR_INVALID_ARG;
+  if (!aligned(m.W, w_align) || !aligned(m.Wq_packed, 16)) return HQQ_ERR_ALIGNMENT;
+  const size_t msz = dtype_size(prm.meta_dtype);
+  if (!aligned(m.scale, msz) || !aligned(m.zero, msz)) return HQQ_ERR_ALIGNMENT;
+  (void)out_dtype;
+  return HQQ_OK;
+}
+
+static hqq_status check_batch_params(const hqq_matrix* mats, int n, const hqq_params* prm) {
+  if (!prm || n < 0 || (n > 0 && !mats)) return HQQ_ERR_INVALID_ARG;
+  if (!nbits_ok(prm->nbits) || !group_ok(prm->group_size) || (prm->axis != 0 && prm->axis != 1))
+    return HQQ_ERR_UNSUPPORTED;
+  if (!wdtype_ok(prm->w_dtype) || !wdtype_ok(prm->meta_dtype)) return HQQ_ERR_UNSUPPORTED;
+  if (prm->quant_scale || prm->quant_zero) return HQQ_ERR_UNSUPPORTED;
+  return HQQ_OK;
+}
+
+HQQ_EXPORT hqq_status hqq_quantize_batched(const hqq_matrix* mats, int n, const hqq_params* prm,
+                                           cudaStream_t stream) {
+  hqq_status st = check_batch_params(mats, n, prm);
+  if (st != HQQ_OK) return st;
+  if ((st = check_solver(prm->iters, prm->p, prm->beta0, prm->kappa)) != HQQ_OK) return st;
+  std::vector<hqqk::QuantJob> jobs;
+  jobs.reserve((size_t)n);
+  for (int i = 0; i < n; ++i) {
+    const hqq_matrix& m = mats[i];
+    if ((st = check_matrix(m, *prm, 16, -1)) != HQQ_OK) return st;
+    if (m.rows * m.cols == 0) continue;
+    hqqk::QuantJob j;
+    j.W = m.W;
+    j.rows = m.rows;
+    j.cols = m.cols;
+    j.n_groups = m.rows * m.cols / prm->group_size;
+    j.w_dtype = prm->w_dtype;
+    j.nbits = prm->nbits;
+    j.group_size = prm->group_size;
+    j.axis = prm->axis;
+    j.iters = prm->iters;
+    j.p = prm->p;
+    j.beta0 = prm->beta0;
+    j.kappa = prm->kappa;
+    j.packed = reinterpret_cast<uint8_t*>(m.Wq_packed);
+    j.scale = m.scale;
+    j.zero = m.zero;
+    j.scale_dtype = prm->meta_dtype;
+    j.zero_dtype = prm->meta_dtype;
+    jobs.push_back(j);
+  }
+  if (jobs.empty()) return HQQ_OK;
+  return cuda_status(hqqk::launch_quantize_batched(jobs.data(), (int)jobs.size(), stream));
+}
+
+HQQ_EXPORT hqq_status hqq_dequantize_batched(const hqq_matrix* mats, int n, const hqq_params* prm,
+                                             hqq_dtype out_dtype, cudaStream_t stream) {
+  hqq_status st = check_batch_params(mats, n, prm);
+  if (st != HQQ_OK) return st;
+  if (!wdtype_ok(out_dtype)) return HQQ_ERR_UNSUPPORTED;
+  std::vector<hqqk::DequantJob> jobs;
+  jobs.reserve((size_t)n);
+  for (int i = 0; i < n; ++i) {
+    const hqq_matrix& m = mats[i];
+    if ((st = check_matrix(m, *prm, 16, out_dtype)) != HQQ_OK) return st;
+    if (m.rows * m.cols == 0) continue;
+    hqqk::DequantJob j;
+    j.packed = reinterpret_cast<const uint8_t*>(m.Wq_packed);
+    j.scale = m.scale;
+    j.zero = m.zero;
+    j.scale_mm = nullptr;
+    j.zero_mm = nullptr;
+    j.meta_group_size = 128;
+    j.meta_dtype = prm->meta_dtype;
+    j.rows = m.rows;
+    j.cols = m.cols;
+    j.n_groups = m.rows * m.cols / prm->group_size;
+    j.nbits = prm->nbits;
+    j.group_size = prm->group_size;
+    j.axis = prm->axis;
+    j.out_dtype = out_dtype;
+    j.out = m.W;
+    jobs.push_back(j);
+  }
+  if (jobs.empty()) return HQQ_OK;
+  return cuda_status(hqqk::launch_dequantize_batched(jobs.data(), (int)jobs.size(), stream));
 }
 
 HQQ_EXPORT hqq_status hqq_quantize_meta(const void* meta, hqq_dtype dtype, int64_t n, int group,

@@ -52,6 +52,44 @@ struct DArgs {
   void* out;
 };
 
+// A batch of matrices sharing one configuration, passed by value as kernel parameters (no
+// device allocation): per-matrix pointers and shapes and the prefix sums of their tile
+// counts; a block finds its matrix with a binary search in parameter space.
+template <int MAXB>
+struct DBatch {
+  DArgs c;  // shared settings (meta dtype, run length, group size); pointer fields unused
+  int n;
+  int64_t tile_start[MAXB + 1];
+  const uint8_t* packed[MAXB];
+  const void* scale[MAXB];
+  const void* zero[MAXB];
+  const float* scale_mm[MAXB];
+  const float* zero_mm[MAXB];
+  int64_t rows[MAXB], cols[MAXB];
+  void* out[MAXB];
+};
+
+template <int MAXB>
+__device__ __forceinline__ DArgs batch_args(const DBatch<MAXB>& b, int64_t tile, int64_t* local) {
+  int lo = 0, hi = b.n - 1;  // the last i with tile_start[i] <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (b.tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  DArgs a = b.c;
+  a.packed = b.packed[lo];
+  a.scale = b.scale[lo];
+  a.zero = b.zero[lo];
+  a.scale_mm = b.scale_mm[lo];
+  a.zero_mm = b.zero_mm[lo];
+  a.rows = b.rows[lo];
+  a.cols = b.cols[lo];
+  a.n = a.rows * a.cols;
+  a.out = b.out[lo];
+  *local = tile - b.tile_start[lo];
+  return a;
+}
+
 // Small non-negative integer (< 2^23) to fp32 without a conversion instruction: OR it into
 // the mantissa of 2^23 and subtract 2^23 (exact; stays on the FMA/ALU pipes).
 __device__ __forceinline__ float u2f_small(uint32_t q) {
@@ -147,12 +185,18 @@ __device__ __forceinline__ uint32_t code_in(uint64_t raw, int off, int i) {
 // computes and stores any, keeping that many loads in flight.
 constexpr int kDChunks = HQQ_DQ_CHUNKS;
 
-template <int NB, int OUT_DT>
-__global__ void __launch_bounds__(kDBlock, HQQ_DQ_MINB) dequant_axis1_kernel(const DArgs a) {
-  const int64_t n_chunks = a.n >> 3;
-  const int64_t pass = (int64_t)gridDim.x * kDBlock * kDChunks;
-  for (int64_t c0 = (int64_t)blockIdx.x * kDBlock * kDChunks + threadIdx.x; c0 < n_chunks;
-       c0 += pass) {
+// Elements per tile of the axis-1 kernel (kDChunks chunks of 8 per thread).
+constexpr int64_t kDTile1 = (int64_t)kDBlock * kDChunks * 8;
+
+template <int NB, int OUT_DT, int MAXB>
+__global__ void __launch_bounds__(kDBlock, HQQ_DQ_MINB)
+    dequant_axis1_kernel(const __grid_constant__ DBatch<MAXB> batch) {
+  const int64_t total = batch.tile_start[batch.n];
+  for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+    int64_t local;
+    const DArgs a = batch_args(batch, t, &local);
+    const int64_t n_chunks = a.n >> 3;
+    const int64_t c0 = local * kDBlock * kDChunks + threadIdx.x;
     uint64_t raw[kDChunks];
     int off[kDChunks];
     float sc[kDChunks], zr[kDChunks];
@@ -181,10 +225,16 @@ __global__ void __launch_bounds__(kDBlock, HQQ_DQ_MINB) dequant_axis1_kernel(con
 }
 
 // axis=0 (groups run down columns): element (r, c) is code j = r % G of group
-// g = (r / G)*cols + c. Rows with cols % 8 == 0 take 8 columns per thread.
-template <int NB, int OUT_DT>
-__global__ void __launch_bounds__(kDBlock) dequant_axis0_kernel(const DArgs a) {
-  const int64_t k0 = ((int64_t)blockIdx.x * kDBlock + threadIdx.x) * 8;
+// g = (r / G)*cols + c. Rows with cols % 8 == 0 take 8 columns per thread; a block covers
+// one tile of kDBlock*8 elements of one matrix.
+constexpr int64_t kDTile0 = (int64_t)kDBlock * 8;
+
+template <int NB, int OUT_DT, int MAXB>
+__global__ void __launch_bounds__(kDBlock)
+    dequant_axis0_kernel(const __grid_constant__ DBatch<MAXB> batch) {
+  int64_t local;
+  const DArgs a = batch_args(batch, (int64_t)blockIdx.x, &local);
+  const int64_t k0 = (local * kDBlock + threadIdx.x) * 8;
   if (k0 >= a.n) return;
   const int G = a.group_size;
   if ((a.cols & 7) == 0) {
@@ -227,57 +277,95 @@ static cudaError_t resident_blocks(K kernel, int* out) {
   return e;
 }
 
-template <int NB, int OUT_DT>
-static cudaError_t launch_nb_dt(const DArgs& a, int axis, cudaStream_t st) {
-  const int64_t threads = (a.n + 7) / 8;
-  const int64_t blocks = (threads + kDBlock - 1) / kDBlock;
-  if (blocks == 0) return cudaSuccess;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  if (axis == 1) {
+template <int MAXB>
+static void fill_dbatch(const DequantJob* jobs, int n, int64_t tile_elems, DBatch<MAXB>* b) {
+  const DequantJob& j0 = jobs[0];
+  DArgs& c = b->c;
+  c.packed = nullptr;
+  c.scale = c.zero = nullptr;
+  c.scale_mm = c.zero_mm = nullptr;
+  c.meta_group_size = j0.meta_group_size > 0 ? j0.meta_group_size : 1;
+  c.meta_dtype = j0.meta_dtype;
+  c.rows = c.cols = c.n = 0;
+  c.group_size = j0.group_size;
+  c.log2_group = 0;
+  while ((1 << c.log2_group) < j0.group_size) ++c.log2_group;
+  c.out = nullptr;
+  int64_t tiles = 0;
+  int k = 0;
+  for (int i = 0; i < n; ++i) {
+    const DequantJob& j = jobs[i];
+    const int64_t elems = j.rows * j.cols;
+    if (elems == 0) continue;
+    b->tile_start[k] = tiles;
+    b->packed[k] = j.packed;
+    b->scale[k] = j.scale;
+    b->zero[k] = j.zero;
+    b->scale_mm[k] = j.scale_mm;
+    b->zero_mm[k] = j.zero_mm;
+    b->rows[k] = j.rows;
+    b->cols[k] = j.cols;
+    b->out[k] = j.out;
+    tiles += (elems + tile_elems - 1) / tile_elems;
+    ++k;
+  }
+  b->tile_start[k] = tiles;
+  b->n = k;
+}
+
+template <int NB, int OUT_DT, int MAXB>
+static cudaError_t launch_nb_dt(const DequantJob* jobs, int n, cudaStream_t st) {
+  DBatch<MAXB> b;
+  if (jobs[0].axis == 1) {
+    fill_dbatch<MAXB>(jobs, n, kDTile1, &b);
+    const int64_t tiles = b.tile_start[b.n];
+    if (tiles == 0) return cudaSuccess;
     int resident = 0;
-    const cudaError_t e = resident_blocks(dequant_axis1_kernel<NB, OUT_DT>, &resident);
+    const cudaError_t e = resident_blocks(dequant_axis1_kernel<NB, OUT_DT, MAXB>, &resident);
     if (e != cudaSuccess) return e;
-    int64_t b1 = (threads + (int64_t)kDBlock * kDChunks - 1) / ((int64_t)kDBlock * kDChunks);
-    if (b1 > resident) b1 = resident;
-    dequant_axis1_kernel<NB, OUT_DT><<<(unsigned)b1, kDBlock, 0, st>>>(a);
+    const int64_t blocks = tiles < resident ? tiles : resident;
+    dequant_axis1_kernel<NB, OUT_DT, MAXB><<<(unsigned)blocks, kDBlock, 0, st>>>(b);
   } else {
-    dequant_axis0_kernel<NB, OUT_DT><<<(unsigned)blocks, kDBlock, 0, st>>>(a);
+    fill_dbatch<MAXB>(jobs, n, kDTile0, &b);
+    const int64_t tiles = b.tile_start[b.n];
+    if (tiles == 0) return cudaSuccess;
+    if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+    dequant_axis0_kernel<NB, OUT_DT, MAXB><<<(unsigned)tiles, kDBlock, 0, st>>>(b);
   }
   return cudaGetLastError();
 }
 
-template <int OUT_DT>
-static cudaError_t launch_dt(const DArgs& a, int nbits, int axis, cudaStream_t st) {
-  switch (nbits) {
-    case 1: return launch_nb_dt<1, OUT_DT>(a, axis, st);
-    case 2: return launch_nb_dt<2, OUT_DT>(a, axis, st);
-    case 3: return launch_nb_dt<3, OUT_DT>(a, axis, st);
-    case 4: return launch_nb_dt<4, OUT_DT>(a, axis, st);
-    default: return launch_nb_dt<8, OUT_DT>(a, axis, st);
+template <int OUT_DT, int MAXB>
+static cudaError_t launch_dt(const DequantJob* jobs, int n, cudaStream_t st) {
+  switch (jobs[0].nbits) {
+    case 1: return launch_nb_dt<1, OUT_DT, MAXB>(jobs, n, st);
+    case 2: return launch_nb_dt<2, OUT_DT, MAXB>(jobs, n, st);
+    case 3: return launch_nb_dt<3, OUT_DT, MAXB>(jobs, n, st);
+    case 4: return launch_nb_dt<4, OUT_DT, MAXB>(jobs, n, st);
+    default: return launch_nb_dt<8, OUT_DT, MAXB>(jobs, n, st);
+  }
+}
+
+template <int MAXB>
+static cudaError_t launch_dq(const DequantJob* jobs, int n, cudaStream_t st) {
+  switch (jobs[0].out_dtype) {
+    case kF16: return launch_dt<kF16, MAXB>(jobs, n, st);
+    case kBF16: return launch_dt<kBF16, MAXB>(jobs, n, st);
+    default: return launch_dt<kF32, MAXB>(jobs, n, st);
   }
 }
 
 cudaError_t launch_dequantize(const DequantJob& j, cudaStream_t st) {
-  DArgs a;
-  a.packed = j.packed;
-  a.scale = j.scale;
-  a.zero = j.zero;
-  a.scale_mm = j.scale_mm;
-  a.zero_mm = j.zero_mm;
-  a.meta_group_size = j.meta_group_size > 0 ? j.meta_group_size : 1;
-  a.meta_dtype = j.meta_dtype;
-  a.rows = j.rows;
-  a.cols = j.cols;
-  a.n = j.rows * j.cols;
-  a.group_size = j.group_size;
-  a.log2_group = 0;
-  while ((1 << a.log2_group) < j.group_size) ++a.log2_group;
-  a.out = j.out;
-  switch (j.out_dtype) {
-    case kF16: return launch_dt<kF16>(a, j.nbits, j.axis, st);
-    case kBF16: return launch_dt<kBF16>(a, j.nbits, j.axis, st);
-    default: return launch_dt<kF32>(a, j.nbits, j.axis, st);
+  return launch_dq<1>(&j, 1, st);
+}
+
+cudaError_t launch_dequantize_batched(const DequantJob* jobs, int n, cudaStream_t st) {
+  for (int i = 0; i < n; i += kMaxBatch) {
+    const int k = n - i < kMaxBatch ? n - i : kMaxBatch;
+    const cudaError_t e = launch_dq<kMaxBatch>(jobs + i, k, st);
+    if (e != cudaSuccess) return e;
   }
+  return cudaSuccess;
 }
 
 // ------------------------------------------------------------------ second level

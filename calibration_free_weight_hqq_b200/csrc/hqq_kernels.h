@@ -38,8 +38,16 @@ struct DequantJob {
   void* out;
 };
 
+// Matrices per batched launch (their pointers and tile prefix sums travel as kernel
+// parameters); larger batches are split into several launches.
+constexpr int kMaxBatch = 256;
+
 cudaError_t launch_quantize(const QuantJob& job, cudaStream_t stream);
+// All jobs share nbits, group_size, axis, iters, p, beta0, kappa and the dtypes.
+cudaError_t launch_quantize_batched(const QuantJob* jobs, int n, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantJob& job, cudaStream_t stream);
+// All jobs share the settings and dtypes; only pointers and shapes differ.
+cudaError_t launch_dequantize_batched(const DequantJob* jobs, int n, cudaStream_t stream);
 cudaError_t launch_quantize_meta(const void* meta, int dtype, int64_t n, int group, uint8_t* q,
                                  float* mm, cudaStream_t stream);
 cudaError_t launch_dequantize_meta(const uint8_t* q, const float* mm, int64_t n, int group,

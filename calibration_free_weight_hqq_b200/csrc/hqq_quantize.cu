@@ -351,18 +351,55 @@ __device__ __forceinline__ float shrink_cutoff_lower_bound(const QArgs& a) {
   return __shfl_sync(0xffffffffu, athr, 0);
 }
 
-// One block solves a tile of NGB consecutive groups. Blocks are short (tens of us) and many,
-// so resident blocks sit at different phases and the MUFU stays fed through each block's
-// load / min-max / packing phases.
-template <int G, int L, int AXIS, int WDT, bool PACK3>
-__global__ void __launch_bounds__(kQBlock, HQQ_MINB) quantize_kernel(const QArgs a) {
+// A batch of matrices sharing one configuration, passed by value as kernel parameters
+// (no device allocation): per-matrix pointers and shapes, and the prefix sums of their
+// tile counts, so that a block finds its matrix with a binary search in parameter space.
+template <int MAXB>
+struct QBatch {
+  QArgs c;                         // shared settings; pointers/shape fields unused
+  int n;                           // matrices in this launch
+  int64_t tile_start[MAXB + 1];    // tile_start[i] = first tile of matrix i
+  const void* W[MAXB];
+  int64_t cols[MAXB], n_groups[MAXB];
+  uint8_t* packed[MAXB];
+  void* scale[MAXB];
+  void* zero[MAXB];
+};
+
+template <int MAXB>
+__device__ __forceinline__ int find_matrix(const QBatch<MAXB>& b, int64_t tile) {
+  int lo = 0, hi = b.n - 1;  // the last i with tile_start[i] <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (b.tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// One block solves a tile of NGB consecutive groups of one matrix. Blocks are short (tens of
+// us) and many, so resident blocks sit at different phases and the MUFU stays fed through
+// each block's load / min-max / packing phases (a persistent grid-stride variant, where all
+// warps of an SM reach those phases together, measured 28 % slower).
+template <int G, int L, int AXIS, int WDT, bool PACK3, int MAXB>
+__global__ void __launch_bounds__(kQBlock, HQQ_MINB)
+    quantize_kernel(const __grid_constant__ QBatch<MAXB> batch) {
   constexpr int E = G / L;
   constexpr int NGB = kQBlock / L;  // groups per block
   __shared__ uint8_t s_codes[PACK3 ? NGB * G : 1];
 
+  const int mi = MAXB == 1 ? 0 : find_matrix(batch, (int64_t)blockIdx.x);
+  const int64_t tile = (int64_t)blockIdx.x - batch.tile_start[mi];
+  QArgs a = batch.c;
+  a.W = batch.W[mi];
+  a.cols = batch.cols[mi];
+  a.n_groups = batch.n_groups[mi];
+  a.packed = batch.packed[mi];
+  a.scale = batch.scale[mi];
+  a.zero = batch.zero[mi];
+
   const int tid = threadIdx.x;
   const int lane = tid % L;
-  const int64_t g = (int64_t)blockIdx.x * NGB + tid / L;
+  const int64_t g = tile * NGB + tid / L;
   const bool valid = g < a.n_groups;
   const unsigned wmask = __ballot_sync(0xffffffffu, valid);  // live lanes of this warp
   const unsigned gmask = L == 1 ? 0u : (((1u << L) - 1u) << ((tid & 31) & ~(L - 1)));
@@ -396,7 +433,7 @@ __global__ void __launch_bounds__(kQBlock, HQQ_MINB) quantize_kernel(const QArgs
   if constexpr (PACK3) {
     // 10 codes of 3 bits per little-endian word; this block's codes start on a word.
     __syncthreads();
-    const int64_t code_base = (int64_t)blockIdx.x * NGB * G;
+    const int64_t code_base = tile * NGB * G;
     const int64_t left = a.n_groups * G - code_base;
     const int n_valid = (int)(left < (int64_t)NGB * G ? left : (int64_t)NGB * G);
     const int n_words = (n_valid + 9) / 10;
@@ -417,63 +454,101 @@ __global__ void __launch_bounds__(kQBlock, HQQ_MINB) quantize_kernel(const QArgs
 #define HQQ_G64_LANES 2
 #endif
 
-template <int G, int L, int AXIS, int WDT>
-static cudaError_t launch_g(const QArgs& a, bool pack3, cudaStream_t st) {
+template <int MAXB>
+static cudaError_t fill_batch(const QuantJob* jobs, int n, int ngb, QBatch<MAXB>* b,
+                              int64_t* tiles_out) {
+  const QuantJob& j0 = jobs[0];
+  QArgs& c = b->c;
+  c.W = nullptr;
+  c.rows = c.cols = c.n_groups = 0;
+  c.nbits = j0.nbits;
+  c.iters = j0.iters;
+  c.qmax = (float)((1 << j0.nbits) - 1);
+  c.p = j0.p;
+  c.beta0 = j0.beta0;
+  c.kappa = j0.kappa;
+  c.packed = nullptr;
+  c.scale = c.zero = nullptr;
+  c.scale_dtype = j0.scale_dtype;
+  c.zero_dtype = j0.zero_dtype;
+  int64_t tiles = 0;
+  int k = 0;
+  for (int i = 0; i < n; ++i) {
+    const QuantJob& j = jobs[i];
+    if (j.n_groups == 0) continue;
+    b->tile_start[k] = tiles;
+    b->W[k] = j.W;
+    b->cols[k] = j.cols;
+    b->n_groups[k] = j.n_groups;
+    b->packed[k] = j.packed;
+    b->scale[k] = j.scale;
+    b->zero[k] = j.zero;
+    tiles += (j.n_groups + ngb - 1) / ngb;
+    ++k;
+  }
+  b->tile_start[k] = tiles;
+  b->n = k;
+  *tiles_out = tiles;
+  return tiles > 0x7fffffffLL ? cudaErrorInvalidValue : cudaSuccess;
+}
+
+template <int G, int L, int AXIS, int WDT, int MAXB>
+static cudaError_t launch_g(const QuantJob* jobs, int n, cudaStream_t st) {
   constexpr int NGB = kQBlock / L;
-  const int64_t blocks = (a.n_groups + NGB - 1) / NGB;
-  if (blocks == 0) return cudaSuccess;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  if (pack3) {
-    quantize_kernel<G, L, AXIS, WDT, true><<<(unsigned)blocks, kQBlock, 0, st>>>(a);
+  QBatch<MAXB> b;
+  int64_t tiles = 0;
+  cudaError_t e = fill_batch<MAXB>(jobs, n, NGB, &b, &tiles);
+  if (e != cudaSuccess) return e;
+  if (tiles == 0) return cudaSuccess;
+  if (jobs[0].nbits == 3) {
+    quantize_kernel<G, L, AXIS, WDT, true, MAXB><<<(unsigned)tiles, kQBlock, 0, st>>>(b);
   } else {
-    quantize_kernel<G, L, AXIS, WDT, false><<<(unsigned)blocks, kQBlock, 0, st>>>(a);
+    quantize_kernel<G, L, AXIS, WDT, false, MAXB><<<(unsigned)tiles, kQBlock, 0, st>>>(b);
   }
   return cudaGetLastError();
 }
 
-template <int AXIS, int WDT>
-static cudaError_t launch_axis_dt(const QArgs& a, int G, bool pack3, cudaStream_t st) {
-  switch (G) {
-    case 8: return launch_g<8, 1, AXIS, WDT>(a, pack3, st);
-    case 16: return launch_g<16, 1, AXIS, WDT>(a, pack3, st);
-    case 32: return launch_g<32, 1, AXIS, WDT>(a, pack3, st);
-    case 64: return launch_g<64, HQQ_G64_LANES, AXIS, WDT>(a, pack3, st);
-    case 128: return launch_g<128, 2 * HQQ_G64_LANES, AXIS, WDT>(a, pack3, st);
-    case 256: return launch_g<256, 4 * HQQ_G64_LANES, AXIS, WDT>(a, pack3, st);
+template <int AXIS, int WDT, int MAXB>
+static cudaError_t launch_axis_dt(const QuantJob* jobs, int n, cudaStream_t st) {
+  switch (jobs[0].group_size) {
+    case 8: return launch_g<8, 1, AXIS, WDT, MAXB>(jobs, n, st);
+    case 16: return launch_g<16, 1, AXIS, WDT, MAXB>(jobs, n, st);
+    case 32: return launch_g<32, 1, AXIS, WDT, MAXB>(jobs, n, st);
+    case 64: return launch_g<64, HQQ_G64_LANES, AXIS, WDT, MAXB>(jobs, n, st);
+    case 128: return launch_g<128, 2 * HQQ_G64_LANES, AXIS, WDT, MAXB>(jobs, n, st);
+    case 256: return launch_g<256, 4 * HQQ_G64_LANES, AXIS, WDT, MAXB>(jobs, n, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_quantize(const QuantJob& j, cudaStream_t st) {
-  QArgs a;
-  a.W = j.W;
-  a.rows = j.rows;
-  a.cols = j.cols;
-  a.n_groups = j.n_groups;
-  a.nbits = j.nbits;
-  a.iters = j.iters;
-  a.qmax = (float)((1 << j.nbits) - 1);
-  a.p = j.p;
-  a.beta0 = j.beta0;
-  a.kappa = j.kappa;
-  a.packed = j.packed;
-  a.scale = j.scale;
-  a.zero = j.zero;
-  a.scale_dtype = j.scale_dtype;
-  a.zero_dtype = j.zero_dtype;
-  const bool pack3 = j.nbits == 3;
+template <int MAXB>
+static cudaError_t launch_batch(const QuantJob* jobs, int n, cudaStream_t st) {
+  const QuantJob& j = jobs[0];
   if (j.axis == 1) {
     switch (j.w_dtype) {
-      case kF16: return launch_axis_dt<1, kF16>(a, j.group_size, pack3, st);
-      case kBF16: return launch_axis_dt<1, kBF16>(a, j.group_size, pack3, st);
-      default: return launch_axis_dt<1, kF32>(a, j.group_size, pack3, st);
+      case kF16: return launch_axis_dt<1, kF16, MAXB>(jobs, n, st);
+      case kBF16: return launch_axis_dt<1, kBF16, MAXB>(jobs, n, st);
+      default: return launch_axis_dt<1, kF32, MAXB>(jobs, n, st);
     }
   }
   switch (j.w_dtype) {
-    case kF16: return launch_axis_dt<0, kF16>(a, j.group_size, pack3, st);
-    case kBF16: return launch_axis_dt<0, kBF16>(a, j.group_size, pack3, st);
-    default: return launch_axis_dt<0, kF32>(a, j.group_size, pack3, st);
+    case kF16: return launch_axis_dt<0, kF16, MAXB>(jobs, n, st);
+    case kBF16: return launch_axis_dt<0, kBF16, MAXB>(jobs, n, st);
+    default: return launch_axis_dt<0, kF32, MAXB>(jobs, n, st);
   }
+}
+
+cudaError_t launch_quantize(const QuantJob& j, cudaStream_t st) {
+  return launch_batch<1>(&j, 1, st);
+}
+
+cudaError_t launch_quantize_batched(const QuantJob* jobs, int n, cudaStream_t st) {
+  for (int i = 0; i < n; i += kMaxBatch) {
+    const int k = n - i < kMaxBatch ? n - i : kMaxBatch;
+    const cudaError_t e = launch_batch<kMaxBatch>(jobs + i, k, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace hqqk

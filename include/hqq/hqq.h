@@ -206,6 +206,33 @@ hqq_status hqq_dequantize_ex(const void* Wq_packed, const void* scale, const voi
                              const hqq_params* params, hqq_dtype out_dtype, void* W_out,
                              cudaStream_t stream);
 
+/* One matrix of a batched call. */
+typedef struct {
+  void* W;          /* device, row-major [rows, cols]: quantize reads it (params->w_dtype);
+                       dequantize writes it (out_dtype). 16-byte aligned. */
+  int64_t rows, cols;
+  void* Wq_packed;  /* device, hqq_packed_bytes(rows, cols, ...) bytes, 16-byte aligned */
+  void* scale;      /* device, rows*cols/group_size values of params->meta_dtype */
+  void* zero;       /* device, likewise */
+} hqq_matrix;
+
+/* Quantize n matrices that share one configuration (params: nbits, group_size, axis, solver
+ * constants, w_dtype, meta_dtype; quant_scale/quant_zero must be 0) with as few launches as
+ * possible: up to 256 matrices per launch, their pointers and shapes passed as kernel
+ * parameters, so one tail instead of one per matrix and no device allocation. Shapes may
+ * differ. Each matrix's results are identical to hqq_quantize_ex on it alone. This is the
+ * whole-model driver: a model with per-layer configurations ("HQQ tutorial"
+ * (devpress.csdn.net) §4.2 layer_configs; "HQQ calibration-free guide" (lnwmold.com) §3.4)
+ * makes one call per configuration. mats: host array of n descriptors (copied before the
+ * call returns). Every matrix is validated before anything is launched. */
+hqq_status hqq_quantize_batched(const hqq_matrix* mats, int n, const hqq_params* params,
+                                cudaStream_t stream);
+
+/* Dequantize n matrices of one configuration into their W fields (out_dtype), batched like
+ * hqq_quantize_batched; results identical to hqq_dequantize_ex per matrix. */
+hqq_status hqq_dequantize_batched(const hqq_matrix* mats, int n, const hqq_params* params,
+                                  hqq_dtype out_dtype, cudaStream_t stream);
+
 /* Second level on its own: 8-bit min/max round-to-nearest of n fp32/f16/bf16 values `meta`
  * (device) in runs of `group` values ("HQQ tutorial" (devpress.csdn.net) §3.3). Per run:
  * step2 = (max-min)/255, s2 = 255/(max-min) (both 1 when max == min), zero2 = -min*s2,

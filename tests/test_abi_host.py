@@ -128,3 +128,21 @@ def test_binding_has_no_cpu_path():
     W = torch.zeros(64, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         hqq.hqq_quantize(W)
+
+
+def test_batched_calls_validate_before_launch(L):
+    m = hqq.HQQMatrix(FAKE, 64, 128, FAKE, FAKE, FAKE)
+    bad = hqq.HQQMatrix(FAKE, 64, 100, FAKE, FAKE, FAKE)   # cols not a multiple of 64
+    arr = (hqq.HQQMatrix * 2)(m, bad)
+    p = hqq.make_params()
+    assert L.hqq_quantize_batched(arr, 2, ctypes.byref(p), None) == SHAPE
+    assert L.hqq_dequantize_batched(arr, 2, ctypes.byref(p), 1, None) == SHAPE
+    assert L.hqq_quantize_batched(None, 3, ctypes.byref(p), None) == INVALID
+    assert L.hqq_quantize_batched(arr, -1, ctypes.byref(p), None) == INVALID
+    q = hqq.make_params(quant_scale=True)
+    assert L.hqq_quantize_batched(arr, 1, ctypes.byref(q), None) == UNSUPPORTED
+    empty = (hqq.HQQMatrix * 1)(hqq.HQQMatrix(None, 0, 128, None, None, None))
+    assert L.hqq_quantize_batched(empty, 1, ctypes.byref(p), None) == OK
+    assert L.hqq_quantize_batched(arr, 0, ctypes.byref(p), None) == OK
+    odd = (hqq.HQQMatrix * 1)(hqq.HQQMatrix(FAKE + 8, 64, 128, FAKE, FAKE, FAKE))
+    assert L.hqq_quantize_batched(odd, 1, ctypes.byref(p), None) == ALIGN
