@@ -231,6 +231,9 @@ def run_ours(args, rank, world, dev):
         "clocks": clocks,
         "gpu_launches": 2 * n_q * args.steps,
     }
+    if not args.per_matrix:
+        res["fixed_point_stop"] = run_fixed_point(hqq, wl, Ws, outs, deqs, params, shapes,
+                                                  stream, args)
     if rank == 0 and not args.no_e2e:
         res["e2e"] = run_e2e(hqq, wl, Ws, outs, dev, args)
     if rank == 0 and not args.no_cpu_baseline:
@@ -242,10 +245,38 @@ def solver_source_digest() -> str:
     """sha1 of the solver's sources, to tell whether a recorded capture is still current."""
     import hashlib
     h = hashlib.sha1()
-    for f in ("hqq_quantize.cu", "hqq_device.cuh"):
+    for f in ("hqq_quantize.cu", "hqq_quantize_impl.cuh", "hqq_device.cuh"):
         with open(os.path.join(HERE, "calibration_free_weight_hqq_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
+
+
+def run_fixed_point(hqq, wl, Ws, outs, deqs, params, shapes, stream, args):
+    """The same step with HQQ_FLAG_STOP_AT_FIXED_POINT (bit-identical results; a warp stops
+    once every remaining evaluation of its groups would repeat the last one). Reported beside
+    the headline, not as it: the work done then depends on the data."""
+    import ctypes
+    fp = hqq.HQQParams.from_buffer_copy(params)
+    fp.flags = hqq.HQQ_FLAG_STOP_AT_FIXED_POINT
+    qb, db = hqq.matrix_batch(Ws, outs), hqq.matrix_batch(deqs, outs)
+
+    def step():
+        hqq.hqq_quantize_batched(Ws, fp, outs=outs, batch=qb, stream=stream)
+        hqq.hqq_dequantize_batched(outs, shapes, fp, W_out=deqs, batch=db, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    return {"value": round(wl.weights / (ms * 1e-3) / 1e9, 3), "unit": UNIT,
+            "ms_per_step": round(ms, 3), "flag": "HQQ_FLAG_STOP_AT_FIXED_POINT",
+            "results": "bit-identical to the headline run (tests/test_gpu_fixed_point.py)"}
 
 
 def _traffic_per_launch(avg_weights):
@@ -417,6 +448,38 @@ def probe_sfu():
     return res
 
 
+def probe_hbm(gib: float = 1.0):
+    """HBM bandwidth for read-only, write-only and copy traffic (16-byte accesses, grid of
+    SMs x 8 blocks of 256 threads), on a buffer of `gib` GiB (far above L2)."""
+    import ctypes
+    L = ctypes.CDLL(os.path.join(HERE, "calibration_free_weight_hqq_b200", "libhqq_probe.so"))
+    L.hqq_probe_hbm.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    blocks, threads = sms * 8, 256
+    nbytes = int(gib * (1 << 30)) // 16 * 16
+    a = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    b = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    sink = torch.empty(blocks * threads, dtype=torch.int32, device="cuda")
+    st = torch.cuda.current_stream()
+    res = {"probe": "hbm", "bytes": nbytes}
+    for op, name, moved in ((0, "write", nbytes), (1, "read", nbytes), (2, "copy", 2 * nbytes)):
+        dst = sink if op == 1 else b
+        for _ in range(3):
+            assert L.hqq_probe_hbm(op, a.data_ptr(), dst.data_ptr(), nbytes, blocks, threads,
+                                   st.cuda_stream) == 0
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(10):
+            L.hqq_probe_hbm(op, a.data_ptr(), dst.data_ptr(), nbytes, blocks, threads,
+                            st.cuda_stream)
+        e1.record(st)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / 10
+        res[name] = {"ms": round(ms, 4), "GB_per_s": round(moved / ms / 1e6, 1)}
+    return res
+
+
 def single(kind: str, reps: int = 10):
     """One [16384, 8192] bf16 matrix (134M weights, 268 MB: larger than L2), 4-bit g64:
     time `reps` solver or dequantize launches after warm-up (the small case the ncu
@@ -459,11 +522,16 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--probe-sfu", action="store_true",
                     help="measure the lg2/ex2 issue rate behind the roofline peak and exit")
+    ap.add_argument("--probe-hbm", action="store_true",
+                    help="measure HBM read-only, write-only and copy bandwidth and exit")
     ap.add_argument("--single", choices=["quantize", "dequantize"],
                     help="time one [16384,8192] matrix (the profiling case) and exit")
     args = ap.parse_args()
     if args.probe_sfu:
         print(json.dumps(probe_sfu()), flush=True)
+        return
+    if args.probe_hbm:
+        print(json.dumps(probe_hbm()), flush=True)
         return
     if args.single:
         print(json.dumps(single(args.single)), flush=True)

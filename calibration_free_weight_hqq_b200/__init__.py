@@ -62,7 +62,10 @@ class HQQParams(ctypes.Structure):
                 ("iters", ctypes.c_int), ("p", ctypes.c_float), ("beta0", ctypes.c_float),
                 ("kappa", ctypes.c_float), ("w_dtype", ctypes.c_int),
                 ("meta_dtype", ctypes.c_int), ("quant_scale", ctypes.c_int),
-                ("quant_zero", ctypes.c_int), ("meta_group_size", ctypes.c_int)]
+                ("quant_zero", ctypes.c_int), ("meta_group_size", ctypes.c_int),
+                ("flags", ctypes.c_int)]
+
+HQQ_FLAG_STOP_AT_FIXED_POINT = 1
 
 
 def library_path() -> str:
@@ -155,11 +158,12 @@ def _meta_shape(rows: int, cols: int, group_size: int, axis: int):
 
 def make_params(nbits=4, group_size=64, axis=1, iters=20, p=0.7, beta0=10.0, kappa=1.01,
                 w_dtype=torch.bfloat16, meta_dtype=None, quant_scale=False, quant_zero=False,
-                meta_group_size=128) -> HQQParams:
+                meta_group_size=128, stop_at_fixed_point=False) -> HQQParams:
     meta_dtype = w_dtype if meta_dtype is None else meta_dtype
     return HQQParams(nbits, group_size, axis, iters, p, beta0, kappa, _TORCH_DT[w_dtype],
                      _TORCH_DT[meta_dtype], int(bool(quant_scale)), int(bool(quant_zero)),
-                     meta_group_size)
+                     meta_group_size,
+                     HQQ_FLAG_STOP_AT_FIXED_POINT if stop_at_fixed_point else 0)
 
 
 def hqq_workspace_bytes(rows: int, cols: int, params: HQQParams) -> int:

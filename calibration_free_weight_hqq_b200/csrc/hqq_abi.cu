@@ -48,6 +48,8 @@ hqq_status check_shape(int64_t rows, int64_t cols, int nbits, int group_size, in
   return HQQ_OK;
 }
 
+bool flags_ok(int flags) { return (flags & ~HQQ_FLAG_STOP_AT_FIXED_POINT) == 0; }
+
 hqq_status check_solver(int iters, float p, float beta0, float kappa) {
   if (iters < 0 || iters > HQQ_MAX_ITERS) return HQQ_ERR_INVALID_ARG;
   if (!(p > 0.0f && p <= 1.0f)) return HQQ_ERR_INVALID_ARG;
@@ -118,6 +120,7 @@ static hqq_status quantize_impl(const void* W, int64_t rows, int64_t cols, const
   hqq_status st = check_shape(rows, cols, prm.nbits, prm.group_size, prm.axis);
   if (st != HQQ_OK) return st;
   if ((st = check_solver(prm.iters, prm.p, prm.beta0, prm.kappa)) != HQQ_OK) return st;
+  if (!flags_ok(prm.flags)) return HQQ_ERR_INVALID_ARG;
   if (!wdtype_ok(prm.w_dtype) || !wdtype_ok(prm.meta_dtype)) return HQQ_ERR_UNSUPPORTED;
   const bool qs = prm.quant_scale != 0, qz = prm.quant_zero != 0;
   if ((qs || qz) && (st = check_meta_group(prm.meta_group_size)) != HQQ_OK) return st;
@@ -159,6 +162,7 @@ static hqq_status quantize_impl(const void* W, int64_t rows, int64_t cols, const
   j.zero = qz ? static_cast<void*>(ws_zero) : zero;
   j.scale_dtype = qs ? hqqk::kF32 : prm.meta_dtype;
   j.zero_dtype = qz ? hqqk::kF32 : prm.meta_dtype;
+  j.flags = prm.flags;
   if ((st = cuda_status(hqqk::launch_quantize(j, stream))) != HQQ_OK) return st;
   if (qs) {
     st = cuda_status(hqqk::launch_quantize_meta(ws_scale, hqqk::kF32, ng, prm.meta_group_size,
@@ -192,6 +196,7 @@ HQQ_EXPORT hqq_status hqq_quantize(const void* W, hqq_dtype dtype, int64_t rows,
   prm.quant_scale = 0;
   prm.quant_zero = 0;
   prm.meta_group_size = 128;
+  prm.flags = 0;
   return quantize_impl(W, rows, cols, prm, Wq_packed, scale, zero, nullptr, nullptr, nullptr, 0,
                        stream);
 }
@@ -292,6 +297,7 @@ HQQ_EXPORT hqq_status hqq_quantize_batched(const hqq_matrix* mats, int n, const 
   hqq_status st = check_batch_params(mats, n, prm);
   if (st != HQQ_OK) return st;
   if ((st = check_solver(prm->iters, prm->p, prm->beta0, prm->kappa)) != HQQ_OK) return st;
+  if (!flags_ok(prm->flags)) return HQQ_ERR_INVALID_ARG;
   std::vector<hqqk::QuantJob> jobs;
   jobs.reserve((size_t)n);
   for (int i = 0; i < n; ++i) {
@@ -316,6 +322,7 @@ HQQ_EXPORT hqq_status hqq_quantize_batched(const hqq_matrix* mats, int n, const 
     j.zero = m.zero;
     j.scale_dtype = prm->meta_dtype;
     j.zero_dtype = prm->meta_dtype;
+    j.flags = prm->flags;
     jobs.push_back(j);
   }
   if (jobs.empty()) return HQQ_OK;

@@ -30,6 +30,9 @@ constexpr int kDBlock = 256;
 #ifndef HQQ_DQ_MINB
 #define HQQ_DQ_MINB 8
 #endif
+#ifndef HQQ_DQ_PREFETCH
+#define HQQ_DQ_PREFETCH 1
+#endif
 
 template <typename T>
 __device__ __forceinline__ void st_out(T* p, const T& v) {
@@ -188,39 +191,75 @@ constexpr int kDChunks = HQQ_DQ_CHUNKS;
 // Elements per tile of the axis-1 kernel (kDChunks chunks of 8 per thread).
 constexpr int64_t kDTile1 = (int64_t)kDBlock * kDChunks * 8;
 
+// One round of a thread's work: kDChunks chunks of 8 elements of one tile, loaded.
+template <int NB>
+struct DRound {
+  const uint8_t* packed;
+  void* out;
+  int64_t c0, n_chunks, n;
+  uint64_t raw[kDChunks];
+  int off[kDChunks];
+  float sc[kDChunks], zr[kDChunks];
+};
+
+template <int NB, int MAXB>
+__device__ __forceinline__ void load_round(const DBatch<MAXB>& batch, int64_t t, DRound<NB>& r) {
+  int64_t local;
+  const DArgs a = batch_args(batch, t, &local);
+  r.packed = a.packed;
+  r.out = a.out;
+  r.n = a.n;
+  r.n_chunks = a.n >> 3;
+  r.c0 = local * kDBlock * kDChunks + threadIdx.x;
+#pragma unroll
+  for (int i = 0; i < kDChunks; ++i) {
+    const int64_t c = r.c0 + (int64_t)i * kDBlock;
+    if (c < r.n_chunks) {
+      r.raw[i] = codes8_raw<NB>(a.packed, c << 3, a.n, r.off[i]);
+      const int64_t g = (c << 3) >> a.log2_group;
+      r.sc[i] = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g);
+      r.zr[i] = meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g);
+    }
+  }
+}
+
+template <int NB, int OUT_DT>
+__device__ __forceinline__ void finish_round(const DRound<NB>& r) {
+#pragma unroll
+  for (int i = 0; i < kDChunks; ++i) {
+    const int64_t c = r.c0 + (int64_t)i * kDBlock;
+    if (c < r.n_chunks) {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        v[j] = __fmul_rn(__fsub_rn(u2f_small(code_in<NB>(r.raw[i], r.off[i], j)), r.zr[i]), r.sc[i]);
+      store8<OUT_DT>(r.out, c << 3, v);  // n and G are multiples of 8 on this path
+    }
+  }
+}
+
+// Grid-stride over tiles; the loads of a thread's next round are issued before the current
+// round is converted and stored, so load latency overlaps the stores instead of following
+// them.
 template <int NB, int OUT_DT, int MAXB>
 __global__ void __launch_bounds__(kDBlock, HQQ_DQ_MINB)
     dequant_axis1_kernel(const __grid_constant__ DBatch<MAXB> batch) {
   const int64_t total = batch.tile_start[batch.n];
-  for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
-    int64_t local;
-    const DArgs a = batch_args(batch, t, &local);
-    const int64_t n_chunks = a.n >> 3;
-    const int64_t c0 = local * kDBlock * kDChunks + threadIdx.x;
-    uint64_t raw[kDChunks];
-    int off[kDChunks];
-    float sc[kDChunks], zr[kDChunks];
-#pragma unroll
-    for (int i = 0; i < kDChunks; ++i) {
-      const int64_t c = c0 + (int64_t)i * kDBlock;
-      if (c < n_chunks) {
-        raw[i] = codes8_raw<NB>(a.packed, c << 3, a.n, off[i]);
-        const int64_t g = (c << 3) >> a.log2_group;
-        sc[i] = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g);
-        zr[i] = meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kDChunks; ++i) {
-      const int64_t c = c0 + (int64_t)i * kDBlock;
-      if (c < n_chunks) {
-        float v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          v[j] = __fmul_rn(__fsub_rn(u2f_small(code_in<NB>(raw[i], off[i], j)), zr[i]), sc[i]);
-        store8<OUT_DT>(a.out, c << 3, v);  // n and G are multiples of 8 on this path
-      }
-    }
+  int64_t t = blockIdx.x;
+  if (t >= total) return;
+  DRound<NB> cur;
+  load_round<NB>(batch, t, cur);
+  for (; t < total; t += gridDim.x) {
+#if HQQ_DQ_PREFETCH
+    DRound<NB> nxt;
+    const bool more = t + gridDim.x < total;
+    if (more) load_round<NB>(batch, t + gridDim.x, nxt);
+    finish_round<NB, OUT_DT>(cur);
+    if (more) cur = nxt;
+#else
+    finish_round<NB, OUT_DT>(cur);
+    if (t + gridDim.x < total) load_round<NB>(batch, t + gridDim.x, cur);
+#endif
   }
 }
 

@@ -21,6 +21,7 @@ struct QuantJob {
   void* zero;        // device, n_groups values of zero_dtype
   int scale_dtype;   // Dt (kF32 when the second level follows)
   int zero_dtype;
+  int flags;         // HQQ_FLAG_* bits
 };
 
 // One matrix of the dequantize path.

@@ -1,11 +1,13 @@
-// hqq_probe.cu - throughput probe of the special-function unit (MUFU lg2/ex2) on this GPU,
-// the unit that bounds the HQQ solver. Built into a separate library (libhqq_probe.so), not
-// the quantization ABI; bench.py --probe-sfu runs it to justify the roofline's peak.
+// hqq_probe.cu - throughput probes behind the rooflines: the special-function unit (MUFU
+// lg2/ex2, which bounds the HQQ solver) and HBM read-only / write-only / copy bandwidth (the
+// dequantizer writes 4 bytes for every byte it reads at 4 bits). Built into a separate
+// library (libhqq_probe.so), not the quantization ABI; bench.py --probe-sfu / --probe-hbm.
 //
 // Every thread runs 8 independent dependency chains of approximate lg2/ex2 (and nothing
 // else but one FADD/FMUL per step), so the SFU issue rate, not latency, limits the kernel.
 // out must hold blocks*threads floats (one store per thread, so the work is not removed).
 #include <cuda_runtime.h>
+#include <stdint.h>
 
 namespace {
 
@@ -39,7 +41,68 @@ __global__ void sfu_probe_kernel(float* out, int iters) {
   out[(size_t)blockIdx.x * blockDim.x + threadIdx.x] = s;
 }
 
+// HBM probes: 16-byte accesses, 4 per thread per pass in flight, grid-stride.
+__global__ void hbm_write_kernel(uint4* dst, size_t n16) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += 4 * stride) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const size_t j = i + k * stride;
+      if (j < n16) dst[j] = make_uint4((uint32_t)j, 1u, 2u, 3u);
+    }
+  }
+}
+__global__ void hbm_read_kernel(const uint4* src, size_t n16, uint32_t* out) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  uint32_t acc = 0;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const size_t j = i + k * stride;
+      v[k] = j < n16 ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc ^= v[k].x ^ v[k].y ^ v[k].z ^ v[k].w;
+  }
+  out[(size_t)blockIdx.x * blockDim.x + threadIdx.x] = acc;
+}
+__global__ void hbm_copy_kernel(const uint4* src, uint4* dst, size_t n16) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const size_t j = i + k * stride;
+      if (j < n16) v[k] = __ldcs(src + j);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const size_t j = i + k * stride;
+      if (j < n16) dst[j] = v[k];
+    }
+  }
+}
+
 }  // namespace
+
+// op: 0 = write `bytes` to a, 1 = read `bytes` from a (one uint32 per thread to b),
+// 2 = copy `bytes` from a to b. bytes must be a multiple of 16; b must hold blocks*threads
+// uint32 for op 1.
+extern "C" __attribute__((visibility("default"))) int hqq_probe_hbm(int op, void* a, void* b,
+                                                                    size_t bytes, int blocks,
+                                                                    int threads, void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t n16 = bytes / 16;
+  if (op == 0) hbm_write_kernel<<<blocks, threads, 0, st>>>(reinterpret_cast<uint4*>(a), n16);
+  else if (op == 1)
+    hbm_read_kernel<<<blocks, threads, 0, st>>>(reinterpret_cast<const uint4*>(a), n16,
+                                                reinterpret_cast<uint32_t*>(b));
+  else
+    hbm_copy_kernel<<<blocks, threads, 0, st>>>(reinterpret_cast<const uint4*>(a),
+                                                reinterpret_cast<uint4*>(b), n16);
+  return (int)cudaGetLastError();
+}
 
 // op: 0 = ex2 only, 1 = lg2 only, 2 = lg2 then ex2. Returns the cudaError_t of the launch.
 extern "C" __attribute__((visibility("default"))) int hqq_probe_sfu(int op, float* out,

@@ -1,0 +1,526 @@
+// hqq_quantize_impl.cuh - the HQQ solver kernel and its launchers (templates). Included by
+// hqq_quantize.cu (iterations run to the end) and hqq_quantize_stop.cu (iterations stop at a
+// fixed point, HQQ_FLAG_STOP_AT_FIXED_POINT), so that each set compiles in its own unit and
+// the unused option costs the other nothing (a runtime test inside the loop measured 8.7 %).
+#pragma once
+
+#include <math.h>
+
+#include "hqq_device.cuh"
+#include "hqq_kernels.h"
+
+namespace hqqk {
+
+constexpr int kQBlock = 160;  // 5 warps; kQBlock*E codes per block is a multiple of 10
+
+// Tuning knobs (compile-time): minimum resident blocks per SM, and whether to round with
+// the hardware round instruction instead of the magic-number add.
+#ifndef HQQ_MINB
+#define HQQ_MINB 4
+#endif
+#ifndef HQQ_USE_FRND
+#define HQQ_USE_FRND 0
+#endif
+// 1: keep the scaled weights Ws = w*s in registers; 0: recompute w*s at each use (fewer
+// registers, one more FMA-pipe op per element and evaluation).
+#ifndef HQQ_STORE_WS
+#define HQQ_STORE_WS 1
+#endif
+
+__device__ __forceinline__ float round_even(float v) {
+#if HQQ_USE_FRND
+  return rintf(v);
+#else
+  return rint_magic(v);
+#endif
+}
+
+struct QArgs {
+  const void* W;
+  int64_t rows, cols, n_groups;
+  int nbits, iters;
+  float qmax, p, beta0, kappa;
+  uint8_t* packed;
+  void* scale;
+  void* zero;
+  int scale_dtype, zero_dtype;
+  int flags;  // bit 0: stop a warp's iterations once all its groups sit at a fixed point
+};
+
+template <int L>
+__device__ __forceinline__ float group_sum(float x, unsigned m) {
+#pragma unroll
+  for (int o = 1; o < L; o <<= 1) x += __shfl_xor_sync(m, x, o);
+  return x;
+}
+template <int L>
+__device__ __forceinline__ double group_sum_d(double x, unsigned m) {
+#pragma unroll
+  for (int o = 1; o < L; o <<= 1) x += __shfl_xor_sync(m, x, o);
+  return x;
+}
+template <int L>
+__device__ __forceinline__ float group_min(float x, unsigned m) {
+#pragma unroll
+  for (int o = 1; o < L; o <<= 1) x = fminf(x, __shfl_xor_sync(m, x, o));
+  return x;
+}
+template <int L>
+__device__ __forceinline__ float group_max(float x, unsigned m) {
+#pragma unroll
+  for (int o = 1; o < L; o <<= 1) x = fmaxf(x, __shfl_xor_sync(m, x, o));
+  return x;
+}
+
+// Flat index of element j (0..G) of group g.
+template <int G, int AXIS>
+__device__ __forceinline__ int64_t elem_index(const QArgs& a, int64_t g, int j) {
+  if constexpr (AXIS == 1) {
+    return g * G + j;  // cols is a multiple of G, so groups tile memory contiguously
+  } else {
+    int64_t rb = g / a.cols, c = g - rb * a.cols;
+    return (rb * G + j) * a.cols + c;
+  }
+}
+
+// A lane's E raw weights: fp32, or two 16-bit values per 32-bit register (low half first),
+// widened to fp32 at each use (exact).
+template <int WDT, int E>
+struct WRaw {
+  static constexpr bool kPacked = WDT != kF32;
+  uint32_t u[kPacked ? E / 2 : E];
+  __device__ __forceinline__ float get(int j) const {
+    if constexpr (!kPacked) {
+      return __uint_as_float(u[j]);
+    } else {
+      const uint32_t x = u[j >> 1];
+      if constexpr (WDT == kBF16) {
+        return (j & 1) ? __uint_as_float(x & 0xffff0000u) : __uint_as_float(x << 16);
+      } else {
+        return f16_bits_to_f32((j & 1) ? (x >> 16) : (x & 0xffffu));
+      }
+    }
+  }
+};
+
+// Load this lane's E elements of group g (16-byte vector loads for axis=1; for axis=0 the
+// lanes of a warp hold consecutive columns, so each row access is coalesced).
+template <int G, int E, int AXIS, int WDT>
+__device__ __forceinline__ void load_group(const QArgs& a, int64_t g, int lane, WRaw<WDT, E>& w) {
+  constexpr int PER16 = WDT == kF32 ? 4 : 8;  // elements per 16-byte vector
+  if constexpr (AXIS == 1) {
+    const int64_t base = g * G + (int64_t)lane * E;
+    const char* src = reinterpret_cast<const char*>(a.W) + base * (WDT == kF32 ? 4 : 2);
+#pragma unroll
+    for (int i = 0; i < E / PER16; ++i) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+      w.u[4 * i] = v.x; w.u[4 * i + 1] = v.y; w.u[4 * i + 2] = v.z; w.u[4 * i + 3] = v.w;
+    }
+  } else {
+    const int64_t rb = g / a.cols, c = g - rb * a.cols;
+    const int64_t base = (rb * G + (int64_t)lane * E) * a.cols + c;
+    if constexpr (WDT == kF32) {
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(a.W);
+#pragma unroll
+      for (int j = 0; j < E; ++j) w.u[j] = __ldg(src + base + (int64_t)j * a.cols);
+    } else {
+      const unsigned short* src = reinterpret_cast<const unsigned short*>(a.W);
+#pragma unroll
+      for (int i = 0; i < E / 2; ++i) {
+        const uint32_t lo = __ldg(src + base + (int64_t)(2 * i) * a.cols);
+        const uint32_t hi = __ldg(src + base + (int64_t)(2 * i + 1) * a.cols);
+        w.u[i] = lo | (hi << 16);
+      }
+    }
+  }
+}
+
+// Exact shrinkage sum over this lane's elements, recomputed from memory (rare path).
+// Elements whose residual bound is below athr_lo have We == 0 exactly and are skipped.
+template <int G, int E, int AXIS, int WDT>
+__device__ __noinline__ double shrink_sum_exact(const QArgs& a, int64_t g, int lane, float s,
+                                                float step, float z, float inv_beta,
+                                                float athr_lo) {
+  const float slack = 1e-3f * (fabsf(z) + a.qmax + 1.0f);
+  const float pm1 = a.p - 1.0f;
+  double acc = 0.0;
+#pragma unroll 1
+  for (int j = 0; j < E; ++j) {
+    const float w = load_elem<WDT>(a.W, elem_index<G, AXIS>(a, g, lane * E + j));
+    const float v = __fadd_rn(__fmul_rn(w, s), z);
+    const float q = fminf(fmaxf(rintf(v), 0.0f), a.qmax);
+    const float d = __fsub_rn(v, q);
+    if (step * (fabsf(d) * 1.001f + slack) < athr_lo) continue;
+    const float r = __fsub_rn(w, __fmul_rn(__fsub_rn(q, z), step));
+    const float ar = fabsf(r);
+    if (!(ar > 0.0f)) continue;
+    const float t = powf(ar, pm1);
+    const float m = fmaxf(__fsub_rn(ar, __fmul_rn(t, inv_beta)), 0.0f);
+    acc += (double)copysignf(m, r);
+  }
+  return acc;
+}
+
+// Store E codes of NB bits (NB in {1,2,4,8}) starting at code index code0.
+template <int NB, int E>
+__device__ __forceinline__ void store_codes(uint8_t* packed, int64_t code0, const uint32_t (&q)[E]) {
+  constexpr int BITS = E * NB;
+  uint8_t* dst = packed + code0 * NB / 8;
+  if constexpr (BITS >= 32) {
+    constexpr int NW = BITS / 32;
+    uint32_t w[NW];
+#pragma unroll
+    for (int i = 0; i < NW; ++i) w[i] = 0;
+#pragma unroll
+    for (int j = 0; j < E; ++j) w[(j * NB) / 32] |= q[j] << ((j * NB) % 32);
+    if constexpr (NW % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < NW / 4; ++i)
+        reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    } else if constexpr (NW % 2 == 0) {
+#pragma unroll
+      for (int i = 0; i < NW / 2; ++i) reinterpret_cast<uint2*>(dst)[i] = make_uint2(w[2 * i], w[2 * i + 1]);
+    } else {
+      reinterpret_cast<uint32_t*>(dst)[0] = w[0];
+    }
+  } else {
+    uint32_t w = 0;
+#pragma unroll
+    for (int j = 0; j < E; ++j) w |= q[j] << (j * NB);
+    if constexpr (BITS == 16) {
+      reinterpret_cast<unsigned short*>(dst)[0] = (unsigned short)w;
+    } else {
+      dst[0] = (uint8_t)w;
+    }
+  }
+}
+
+// One evaluation of candidate zero z over this lane's elements: the lp error (four
+// partial sums) and the code sum.
+template <int E, int WDT, bool CLAMP, bool P_ONE>
+__device__ __forceinline__ void evaluate(const float (&ws)[HQQ_STORE_WS ? E : 1],
+                                         const WRaw<WDT, E>& w, float s,
+                                         float z, float step, float qmax, float pp, float& e,
+                                         float& sq) {
+  float ea[4] = {0.f, 0.f, 0.f, 0.f};
+  float qa[2] = {0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < E; ++j) {
+    const float wsj = HQQ_STORE_WS ? ws[j] : __fmul_rn(w.get(j), s);
+    const float v = __fadd_rn(wsj, z);
+    const float q = round_even(CLAMP ? fminf(fmaxf(v, 0.0f), qmax) : v);
+    const float r = __fsub_rn(w.get(j), __fmul_rn(__fsub_rn(q, z), step));
+    const float term = P_ONE ? fabsf(r) : ex2_approx(__fmul_rn(pp, lg2_approx(fabsf(r))));
+    ea[j & 3] = __fadd_rn(ea[j & 3], term);
+    qa[j & 1] += q;
+  }
+  e = __fadd_rn(__fadd_rn(ea[0], ea[1]), __fadd_rn(ea[2], ea[3]));
+  sq = qa[0] + qa[1];
+}
+
+// The solver for the group this lane belongs to, from its raw weights in registers.
+// Returns the group's final codes (this lane's E of them), step and best zero.
+template <int G, int L, int AXIS, int WDT, bool STOP>
+__device__ __forceinline__ void solve_group(const QArgs& a, int64_t g, int lane, unsigned gmask,
+                                            unsigned wmask, float athr_lo,
+                                            const WRaw<WDT, G / L>& w, uint32_t (&q)[G / L],
+                                            float& step_out, float& zbest_out) {
+  constexpr int E = G / L;
+  // ---- min/max round-to-nearest initialisation
+  float mn = w.get(0), mx = w.get(0);
+#pragma unroll
+  for (int j = 1; j < E; ++j) {
+    mn = fminf(mn, w.get(j));
+    mx = fmaxf(mx, w.get(j));
+  }
+  if constexpr (L > 1) {
+    mn = group_min<L>(mn, gmask);
+    mx = group_max<L>(mx, gmask);
+  }
+  const float qmax = a.qmax;
+  float s = 1.0f, step = 1.0f;
+  if (mx > mn) {
+    const float range = __fsub_rn(mx, mn);
+    s = __fdiv_rn(qmax, range);
+    step = __fdiv_rn(range, qmax);
+  }
+  const float z0 = __fmul_rn(-mn, s);
+  float ws[HQQ_STORE_WS ? E : 1];  // scaled weights Ws = w*s, resident for all evaluations
+  double acc = 0.0;
+#pragma unroll
+  for (int j = 0; j < E; ++j) {
+    const float wsj = __fmul_rn(w.get(j), s);
+    if constexpr (HQQ_STORE_WS) ws[j] = wsj;
+    acc = __dadd_rn(acc, f32_to_f64_exact(wsj));
+  }
+  if constexpr (L > 1) acc = group_sum_d<L>(acc, gmask);
+  const double S_ws = (double)(float)acc;  // rounded once to fp32
+  const double s_d = (double)s;
+  const float wsmin = __fmul_rn(mn, s), wsmax = __fmul_rn(mx, s);
+
+  // ---- iterations
+  const float pp = a.p;
+  const bool p_one = pp == 1.0f;  // |r|^1 needs no transcendental (and is then exact)
+  float z = z0, zbest = z0, best = __int_as_float(0x7f800000), beta = a.beta0;
+  for (int k = 0;; ++k) {
+    // Codes stay inside [0, qmax] without clamping iff the group's extreme values do:
+    // rint(v) >= 0 for v >= -0.5 and rint(v) <= qmax for v < qmax + 0.5.
+    const bool inside = __fadd_rn(wsmin, z) >= -0.5f && __fadd_rn(wsmax, z) < qmax + 0.5f;
+    const bool clamp = __any_sync(wmask, !inside);
+    float e, sq;
+    if (p_one) {
+      if (clamp) evaluate<E, WDT, true, true>(ws, w, s, z, step, qmax, pp, e, sq);
+      else evaluate<E, WDT, false, true>(ws, w, s, z, step, qmax, pp, e, sq);
+    } else {
+      if (clamp) evaluate<E, WDT, true, false>(ws, w, s, z, step, qmax, pp, e, sq);
+      else evaluate<E, WDT, false, false>(ws, w, s, z, step, qmax, pp, e, sq);
+    }
+    if constexpr (L > 1) {
+      e = group_sum<L>(e, gmask);
+      sq = group_sum<L>(sq, gmask);
+    }
+    if (e < best) {
+      best = e;
+      zbest = z;
+    }
+    if (k == a.iters) break;
+
+    // Bound on max_j |r_j|: unclamped codes leave |v - Q| <= 1/2, clamped ones at most the
+    // distance of the group's extreme scaled weight from the code range.
+    const float hi = fmaxf(0.5f, fmaxf(-__fadd_rn(wsmin, z), __fsub_rn(__fadd_rn(wsmax, z), qmax)));
+    const float bound = step * (hi * 1.001f + 1e-3f * (fabsf(z) + qmax + 1.0f));
+    double swe = 0.0;
+    const bool no_shrink = bound < athr_lo;  // then also for every later update at this z
+    if (!no_shrink) {
+      swe = shrink_sum_exact<G, E, AXIS, WDT>(a, g, lane, s, step, z, __fdiv_rn(1.0f, beta), athr_lo);
+      if constexpr (L > 1) swe = group_sum_d<L>(swe, gmask);
+    }
+    // Closed-form zero. Every lane computes it (a masked warp instruction costs the pipe as
+    // much as a full one, so one lane computing and broadcasting would only add a shuffle).
+    const double num = __dadd_rn(__dsub_rn(small_int_f32_to_f64(sq), S_ws), __dmul_rn(s_d, swe));
+    const float znew = __double2float_rn(__dmul_rn(num, 1.0 / (double)G));  // G = 2^k: exact
+    beta = __fmul_rn(beta, a.kappa);
+    if constexpr (STOP) {
+      // Fixed point: same zero, provably no shrinkage from here on, so every remaining
+      // evaluation repeats this one exactly (same codes and error, never a new best).
+      const bool settled = no_shrink && __float_as_uint(znew) == __float_as_uint(z);
+      z = znew;
+      if (__all_sync(wmask, settled)) break;
+    } else {
+      z = znew;
+    }
+  }
+
+  // ---- final codes: the integer is read from the low mantissa bits of v + 1.5*2^23
+#pragma unroll
+  for (int j = 0; j < E; ++j) {
+    const float wsj = HQQ_STORE_WS ? ws[j] : __fmul_rn(w.get(j), s);
+    const float v = fminf(fmaxf(__fadd_rn(wsj, zbest), 0.0f), qmax);
+    q[j] = __float_as_uint(__fadd_rn(v, kRoundMagic)) - 0x4B400000u;
+  }
+  step_out = step;
+  zbest_out = zbest;
+}
+
+// Lower bound (absolute units) of the shrinkage cut-off |r| > beta_k^(-1/(2-p)) over all
+// updates: beta_k is non-decreasing, so the last update has the smallest cut-off. Lane 0 of
+// each warp computes it and broadcasts it (it only selects the exact path, never a result).
+__device__ __forceinline__ float shrink_cutoff_lower_bound(const QArgs& a) {
+  float athr = 0.0f;
+  if ((threadIdx.x & 31) == 0 && a.iters > 0) {
+    float b = a.beta0;
+    for (int k = 1; k < a.iters; ++k) b = __fmul_rn(b, a.kappa);
+    athr = powf(__fdiv_rn(1.0f, b), 1.0f / (2.0f - a.p)) * 0.998f;
+  }
+  return __shfl_sync(0xffffffffu, athr, 0);
+}
+
+// A batch of matrices sharing one configuration, passed by value as kernel parameters
+// (no device allocation): per-matrix pointers and shapes, and the prefix sums of their
+// tile counts, so that a block finds its matrix with a binary search in parameter space.
+template <int MAXB>
+struct QBatch {
+  QArgs c;                         // shared settings; pointers/shape fields unused
+  int n;                           // matrices in this launch
+  int64_t tile_start[MAXB + 1];    // tile_start[i] = first tile of matrix i
+  const void* W[MAXB];
+  int64_t cols[MAXB], n_groups[MAXB];
+  uint8_t* packed[MAXB];
+  void* scale[MAXB];
+  void* zero[MAXB];
+};
+
+template <int MAXB>
+__device__ __forceinline__ int find_matrix(const QBatch<MAXB>& b, int64_t tile) {
+  int lo = 0, hi = b.n - 1;  // the last i with tile_start[i] <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (b.tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// One block solves a tile of NGB consecutive groups of one matrix. Blocks are short (tens of
+// us) and many, so resident blocks sit at different phases and the MUFU stays fed through
+// each block's load / min-max / packing phases (a persistent grid-stride variant, where all
+// warps of an SM reach those phases together, measured 28 % slower).
+template <int G, int L, int AXIS, int WDT, bool PACK3, int MAXB, bool STOP>
+__global__ void __launch_bounds__(kQBlock, HQQ_MINB)
+    quantize_kernel(const __grid_constant__ QBatch<MAXB> batch) {
+  constexpr int E = G / L;
+  constexpr int NGB = kQBlock / L;  // groups per block
+  __shared__ uint8_t s_codes[PACK3 ? NGB * G : 1];
+
+  const int mi = MAXB == 1 ? 0 : find_matrix(batch, (int64_t)blockIdx.x);
+  const int64_t tile = (int64_t)blockIdx.x - batch.tile_start[mi];
+  QArgs a = batch.c;
+  a.W = batch.W[mi];
+  a.cols = batch.cols[mi];
+  a.n_groups = batch.n_groups[mi];
+  a.packed = batch.packed[mi];
+  a.scale = batch.scale[mi];
+  a.zero = batch.zero[mi];
+
+  const int tid = threadIdx.x;
+  const int lane = tid % L;
+  const int64_t g = tile * NGB + tid / L;
+  const bool valid = g < a.n_groups;
+  const unsigned wmask = __ballot_sync(0xffffffffu, valid);  // live lanes of this warp
+  const unsigned gmask = L == 1 ? 0u : (((1u << L) - 1u) << ((tid & 31) & ~(L - 1)));
+  const float athr_lo = shrink_cutoff_lower_bound(a);
+
+  if (valid) {
+    WRaw<WDT, E> w;  // raw weights, resident for all evaluations
+    load_group<G, E, AXIS, WDT>(a, g, lane, w);
+    uint32_t q[E];
+    float step, zbest;
+    solve_group<G, L, AXIS, WDT, STOP>(a, g, lane, gmask, wmask, athr_lo, w, q, step, zbest);
+    if (lane == 0) {
+      store_meta(a.scale, a.scale_dtype, g, step);
+      store_meta(a.zero, a.zero_dtype, g, zbest);
+    }
+    const int64_t code0 = g * G + (int64_t)lane * E;
+    if constexpr (PACK3) {
+      uint8_t* sc = s_codes + (tid / L) * G + lane * E;
+#pragma unroll
+      for (int j = 0; j < E; ++j) sc[j] = (uint8_t)q[j];
+    } else {
+      switch (a.nbits) {
+        case 1: store_codes<1, E>(a.packed, code0, q); break;
+        case 2: store_codes<2, E>(a.packed, code0, q); break;
+        case 4: store_codes<4, E>(a.packed, code0, q); break;
+        default: store_codes<8, E>(a.packed, code0, q); break;
+      }
+    }
+  }
+
+  if constexpr (PACK3) {
+    // 10 codes of 3 bits per little-endian word; this block's codes start on a word.
+    __syncthreads();
+    const int64_t code_base = tile * NGB * G;
+    const int64_t left = a.n_groups * G - code_base;
+    const int n_valid = (int)(left < (int64_t)NGB * G ? left : (int64_t)NGB * G);
+    const int n_words = (n_valid + 9) / 10;
+    uint32_t* out = reinterpret_cast<uint32_t*>(a.packed) + code_base / 10;
+    for (int wi = tid; wi < n_words; wi += kQBlock) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int i = 0; i < 10; ++i) {
+        const int idx = wi * 10 + i;
+        if (idx < n_valid) word |= (uint32_t)s_codes[idx] << (3 * i);
+      }
+      out[wi] = word;
+    }
+  }
+}
+
+#ifndef HQQ_G64_LANES
+#define HQQ_G64_LANES 2
+#endif
+
+template <int MAXB>
+static cudaError_t fill_batch(const QuantJob* jobs, int n, int ngb, QBatch<MAXB>* b,
+                              int64_t* tiles_out) {
+  const QuantJob& j0 = jobs[0];
+  QArgs& c = b->c;
+  c.W = nullptr;
+  c.rows = c.cols = c.n_groups = 0;
+  c.nbits = j0.nbits;
+  c.iters = j0.iters;
+  c.qmax = (float)((1 << j0.nbits) - 1);
+  c.p = j0.p;
+  c.beta0 = j0.beta0;
+  c.kappa = j0.kappa;
+  c.packed = nullptr;
+  c.scale = c.zero = nullptr;
+  c.scale_dtype = j0.scale_dtype;
+  c.zero_dtype = j0.zero_dtype;
+  c.flags = j0.flags;
+  int64_t tiles = 0;
+  int k = 0;
+  for (int i = 0; i < n; ++i) {
+    const QuantJob& j = jobs[i];
+    if (j.n_groups == 0) continue;
+    b->tile_start[k] = tiles;
+    b->W[k] = j.W;
+    b->cols[k] = j.cols;
+    b->n_groups[k] = j.n_groups;
+    b->packed[k] = j.packed;
+    b->scale[k] = j.scale;
+    b->zero[k] = j.zero;
+    tiles += (j.n_groups + ngb - 1) / ngb;
+    ++k;
+  }
+  b->tile_start[k] = tiles;
+  b->n = k;
+  *tiles_out = tiles;
+  return tiles > 0x7fffffffLL ? cudaErrorInvalidValue : cudaSuccess;
+}
+
+template <int G, int L, int AXIS, int WDT, int MAXB, bool STOP>
+static cudaError_t launch_g(const QuantJob* jobs, int n, cudaStream_t st) {
+  constexpr int NGB = kQBlock / L;
+  QBatch<MAXB> b;
+  int64_t tiles = 0;
+  cudaError_t e = fill_batch<MAXB>(jobs, n, NGB, &b, &tiles);
+  if (e != cudaSuccess) return e;
+  if (tiles == 0) return cudaSuccess;
+  if (jobs[0].nbits == 3) {
+    quantize_kernel<G, L, AXIS, WDT, true, MAXB, STOP><<<(unsigned)tiles, kQBlock, 0, st>>>(b);
+  } else {
+    quantize_kernel<G, L, AXIS, WDT, false, MAXB, STOP><<<(unsigned)tiles, kQBlock, 0, st>>>(b);
+  }
+  return cudaGetLastError();
+}
+
+template <int AXIS, int WDT, int MAXB, bool STOP>
+static cudaError_t launch_axis_dt(const QuantJob* jobs, int n, cudaStream_t st) {
+  switch (jobs[0].group_size) {
+    case 8: return launch_g<8, 1, AXIS, WDT, MAXB, STOP>(jobs, n, st);
+    case 16: return launch_g<16, 1, AXIS, WDT, MAXB, STOP>(jobs, n, st);
+    case 32: return launch_g<32, 1, AXIS, WDT, MAXB, STOP>(jobs, n, st);
+    case 64: return launch_g<64, HQQ_G64_LANES, AXIS, WDT, MAXB, STOP>(jobs, n, st);
+    case 128: return launch_g<128, 2 * HQQ_G64_LANES, AXIS, WDT, MAXB, STOP>(jobs, n, st);
+    case 256: return launch_g<256, 4 * HQQ_G64_LANES, AXIS, WDT, MAXB, STOP>(jobs, n, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int MAXB, bool STOP>
+static cudaError_t launch_batch(const QuantJob* jobs, int n, cudaStream_t st) {
+  const QuantJob& j = jobs[0];
+  if (j.axis == 1) {
+    switch (j.w_dtype) {
+      case kF16: return launch_axis_dt<1, kF16, MAXB, STOP>(jobs, n, st);
+      case kBF16: return launch_axis_dt<1, kBF16, MAXB, STOP>(jobs, n, st);
+      default: return launch_axis_dt<1, kF32, MAXB, STOP>(jobs, n, st);
+    }
+  }
+  switch (j.w_dtype) {
+    case kF16: return launch_axis_dt<0, kF16, MAXB, STOP>(jobs, n, st);
+    case kBF16: return launch_axis_dt<0, kBF16, MAXB, STOP>(jobs, n, st);
+    default: return launch_axis_dt<0, kF32, MAXB, STOP>(jobs, n, st);
+  }
+}
+
+}  // namespace hqqk

@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define HQQ_ABI_VERSION 1
+#define HQQ_ABI_VERSION 2
 
 typedef enum {
   HQQ_OK = 0,
@@ -96,7 +96,17 @@ typedef struct {
   int quant_scale;      /* nonzero: scale is stored as uint8 codes + fp32 (step2, zero2) */
   int quant_zero;       /* nonzero: zero is stored as uint8 codes + fp32 (step2, zero2) */
   int meta_group_size;  /* run length of the second level (128 in the shipped workloads) */
+  int flags;            /* HQQ_FLAG_* bits (0: none) */
 } hqq_params;
+
+/* Stop a group's iterations once they can only repeat themselves: when an update returns the
+ * zero bit-for-bit unchanged and the group's residual bound proves that the shrinkage stays
+ * zero for every remaining update, every later evaluation reproduces the last one exactly
+ * (same codes, same error, no new best), so the results are bit-identical to running all
+ * iters. Applied per warp of groups (a warp stops when all its groups have settled). Off by
+ * default: with it, the work done depends on the data rather than being iters+1
+ * evaluations per group. */
+#define HQQ_FLAG_STOP_AT_FIXED_POINT 1
 
 /* Number of quantization groups of a [rows, cols] weight: rows*cols/group_size.
  * Returns -1 if the grouped dimension (cols for axis=1, rows for axis=0) is not a multiple

@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(L):
     assert "hqq_quantize" in names and "hqq_dequantize" in names and len(names) >= 12
     for n in names:
         assert hasattr(L, n), n
-    assert L.hqq_abi_version() == 1
+    assert L.hqq_abi_version() == 2
 
 
 def test_size_helpers_match_layout(L):
@@ -146,3 +146,12 @@ def test_batched_calls_validate_before_launch(L):
     assert L.hqq_quantize_batched(arr, 0, ctypes.byref(p), None) == OK
     odd = (hqq.HQQMatrix * 1)(hqq.HQQMatrix(FAKE + 8, 64, 128, FAKE, FAKE, FAKE))
     assert L.hqq_quantize_batched(odd, 1, ctypes.byref(p), None) == ALIGN
+
+
+def test_unknown_flags_are_rejected(L):
+    p = hqq.make_params()
+    p.flags = 2
+    assert L.hqq_quantize_ex(FAKE, 64, 128, ctypes.byref(p), FAKE, FAKE, FAKE, None, None, None,
+                             0, None) == INVALID
+    arr = (hqq.HQQMatrix * 1)(hqq.HQQMatrix(FAKE, 64, 128, FAKE, FAKE, FAKE))
+    assert L.hqq_quantize_batched(arr, 1, ctypes.byref(p), None) == INVALID
