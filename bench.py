@@ -19,6 +19,7 @@ of the same workload and prints the same metric with "impl": "reference".
 
 Multi-GPU (torchrun): weak scaling - every rank quantizes its own model replica (distinct
 seeds); no collective on the data path; the barrier and the max-over-ranks time use NCCL.
+--shard instead splits one model's matrices over the ranks (strong scaling).
 """
 from __future__ import annotations
 
@@ -104,6 +105,35 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- multi-rank helpers
+
+
+def replica_seed_offset(rank: int) -> int:
+    """Weak scaling: rank r quantizes its own model replica, seeded apart from the others."""
+    return rank * 100003
+
+
+def partition_by_weight(sizes, world: int):
+    """Strong scaling (--shard): split matrix indices over ranks, largest first onto the
+    least-loaded rank, so every matrix lands on exactly one rank and loads stay balanced."""
+    loads = [0] * world
+    parts = [[] for _ in range(world)]
+    for i in sorted(range(len(sizes)), key=lambda i: -sizes[i]):
+        r = min(range(world), key=lambda r: loads[r])
+        parts[r].append(i)
+        loads[r] += sizes[i]
+    return [sorted(p) for p in parts]
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank time over all ranks (every rank gets it)."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def build_model(workload, device, seed_offset: int):
     from calibration_free_weight_hqq_b200 import synthetic
     Ws = []
@@ -130,8 +160,11 @@ def run_ours(args, rank, world, dev):
     import calibration_free_weight_hqq_b200 as hqq
     from calibration_free_weight_hqq_b200 import workloads
     wl = workloads.llama7b_model_4b()
+    if args.shard and world > 1:
+        part = partition_by_weight([m.numel for m in wl.matrices], world)[rank]
+        wl = workloads.Workload(wl.name, wl.description, [wl.matrices[i] for i in part])
     mats = wl.matrices
-    Ws = build_model(wl, dev, seed_offset=rank * 100003)
+    Ws = build_model(wl, dev, seed_offset=0 if args.shard else replica_seed_offset(rank))
     outs, deqs = alloc_outputs(hqq, wl, dev)
     stream = torch.cuda.current_stream()
     n_w = wl.weights
@@ -184,14 +217,12 @@ def run_ours(args, rank, world, dev):
             step(evs[k])
         t1.record(stream)
         barrier()
-    ms_total = t0.elapsed_time(t1)
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     q_ms = [e[0].elapsed_time(e[1]) for ev in evs for e in ev]
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
     ms_step = ms_total / args.steps
-    value = world * n_w / (ms_step * 1e-3) / 1e9
+    # weak: every rank did a whole model; strong (--shard): the ranks shared one model
+    total_weights = workloads.llama7b_model_4b().weights if args.shard else world * n_w
+    value = total_weights / (ms_step * 1e-3) / 1e9
 
     # roofline of the dominant kernel (the solver): algorithmic MUFU work per launch over
     # its measured average launch duration
@@ -208,7 +239,8 @@ def run_ours(args, rank, world, dev):
     res = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "strong" if args.shard else "weak",
+        "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded LLM-like bf16 weights: per-row sigma, 0.1% outliers)",
         "config": {"workload": wl.name, "matrices": len(mats), "weights": n_w,
                    "w_dtype": "bf16", "nbits": 4, "group_size": 64, "axis": 1, "iters": 20,
@@ -516,6 +548,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shard", action="store_true",
+                    help="N>1: split one model's matrices over the ranks (strong scaling) "
+                         "instead of one replica per rank (weak scaling, the default)")
     ap.add_argument("--per-matrix", action="store_true",
                     help="one launch per matrix instead of the batched whole-model calls")
     ap.add_argument("--no-cpu-baseline", action="store_true")
