@@ -99,9 +99,13 @@ def lib() -> ctypes.CDLL:
                                                  ctypes.POINTER(HQQParams), i32, P]
             L.hqq_quantize_meta.argtypes = [P, i32, i64, i32, P, P, P]
             L.hqq_dequantize_meta.argtypes = [P, P, i64, i32, P, P]
+            L.hqq_linear.argtypes = [P, i64, i64, i32, P, P, P, P, i64,
+                                     ctypes.POINTER(HQQParams), P, P]
+            L.hqq_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
             for f in ("hqq_quantize", "hqq_dequantize", "hqq_quantize_ex", "hqq_dequantize_ex",
                       "hqq_quantize_meta", "hqq_dequantize_meta", "hqq_quantize_ex_noalloc",
-                      "hqq_quantize_batched", "hqq_dequantize_batched"):
+                      "hqq_quantize_batched", "hqq_dequantize_batched", "hqq_linear",
+                      "hqq_wait_timeouts"):
                 getattr(L, f).restype = i32
             L.hqq_packed_bytes.argtypes = [i64, i64, i32, i32, i32]
             L.hqq_packed_bytes.restype = sz
@@ -363,3 +367,35 @@ def hqq_dequantize_meta(q: torch.Tensor, mm: torch.Tensor, group: int = 128, *, 
                                    _cuda(out, "out"), _stream(stream))
     _check(st, "hqq_dequantize_meta")
     return out
+
+
+def hqq_linear(X: torch.Tensor, Wq_packed: torch.Tensor, scale: torch.Tensor,
+               zero: torch.Tensor, N: int, params: Optional[HQQParams] = None, *,
+               bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """Forward pass of a 4-bit, group-64, axis-1 HQQ linear layer on the tensor cores:
+    Y = X @ W'.T (+ bias), W' = the weight [N, K] dequantized to X's dtype (bf16 or fp16).
+    X is [M, K] (or any [..., K]); scale/zero come from hqq_quantize* of W [N, K]."""
+    if params is None:
+        params = make_params(4, 64, 1, w_dtype=X.dtype, meta_dtype=scale.dtype)
+    lead = X.shape[:-1]
+    K = X.shape[-1]
+    M = 1
+    for d in lead:
+        M *= d
+    X2 = X.reshape(M, K)
+    if Y is None:
+        Y = torch.empty(*lead, N, dtype=X.dtype, device=X.device)
+    st = lib().hqq_linear(_cuda(X2, "X"), M, K, _TORCH_DT.get(X.dtype, -1),
+                          _cuda(Wq_packed, "Wq_packed"), _cuda(scale, "scale"),
+                          _cuda(zero, "zero"), _cuda(bias, "bias") if bias is not None else None,
+                          N, ctypes.byref(params), _cuda(Y, "Y"), _stream(stream))
+    _check(st, "hqq_linear")
+    return Y
+
+
+def hqq_wait_timeouts() -> int:
+    """Bounded in-kernel waits that ran out of time since load (0 on healthy runs)."""
+    n = ctypes.c_uint(0)
+    _check(lib().hqq_wait_timeouts(ctypes.byref(n)), "hqq_wait_timeouts")
+    return int(n.value)

@@ -388,3 +388,47 @@ HQQ_EXPORT hqq_status hqq_dequantize_meta(const void* q_u8, const void* mm, int6
                                                   reinterpret_cast<const float*>(mm), n, group,
                                                   reinterpret_cast<float*>(out_f32), stream));
 }
+
+HQQ_EXPORT hqq_status hqq_linear(const void* X, int64_t M, int64_t K, hqq_dtype x_dtype,
+                                 const void* Wq_packed, const void* scale, const void* zero,
+                                 const void* bias, int64_t N, const hqq_params* params, void* Y,
+                                 cudaStream_t stream) {
+  if (!params) return HQQ_ERR_INVALID_ARG;
+  const hqq_params& prm = *params;
+  if (M < 0 || N < 0 || K < 0) return HQQ_ERR_INVALID_ARG;
+  if (x_dtype != HQQ_BF16 && x_dtype != HQQ_F16) return HQQ_ERR_UNSUPPORTED;
+  if (prm.nbits != 4 || prm.group_size != 64 || prm.axis != 1 || prm.quant_scale ||
+      prm.quant_zero)
+    return HQQ_ERR_UNSUPPORTED;
+  if (!wdtype_ok(prm.meta_dtype)) return HQQ_ERR_INVALID_ARG;
+  if (K % 64 != 0 || N % 8 != 0) return HQQ_ERR_SHAPE;
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) ||
+      (M + 255) / 256 > 65535)
+    return HQQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return HQQ_OK;
+  if (!Y) return HQQ_ERR_INVALID_ARG;
+  if (K > 0 && (!X || !Wq_packed || !scale || !zero)) return HQQ_ERR_INVALID_ARG;
+  if (!aligned(Y, 16) || !aligned(bias, 2)) return HQQ_ERR_ALIGNMENT;
+  if (K > 0 && (!aligned(X, 16) || !aligned(Wq_packed, 16) ||
+                !aligned(scale, dtype_size(prm.meta_dtype)) ||
+                !aligned(zero, dtype_size(prm.meta_dtype))))
+    return HQQ_ERR_ALIGNMENT;
+  hqqk::GemmJob j;
+  j.X = X;
+  j.packed = reinterpret_cast<const uint8_t*>(Wq_packed);
+  j.scale = scale;
+  j.zero = zero;
+  j.bias = bias;
+  j.Y = Y;
+  j.M = M;
+  j.N = N;
+  j.K = K;
+  j.x_dtype = x_dtype;
+  j.meta_dtype = prm.meta_dtype;
+  return cuda_status(hqqk::launch_w4a16_gemm(j, stream));
+}
+
+HQQ_EXPORT hqq_status hqq_wait_timeouts(unsigned int* count) {
+  if (!count) return HQQ_ERR_INVALID_ARG;
+  return cuda_status(hqqk::read_gemm_timeouts(count));
+}

@@ -49,6 +49,25 @@ cudaError_t launch_quantize_batched(const QuantJob* jobs, int n, cudaStream_t st
 cudaError_t launch_dequantize(const DequantJob& job, cudaStream_t stream);
 // All jobs share the settings and dtypes; only pointers and shapes differ.
 cudaError_t launch_dequantize_batched(const DequantJob* jobs, int n, cudaStream_t stream);
+// Y[M, N] = X[M, K] · W'^T (+ bias) with W' the dequantized 4-bit, group-64, axis-1 weight
+// [N, K]; X, bias and Y share x_dtype (kBF16 or kF16). Shapes and alignment are validated by
+// the caller: K % 64 == 0, N % 8 == 0, 16-byte aligned X, packed and Y.
+struct GemmJob {
+  const void* X;
+  const uint8_t* packed;
+  const void* scale;
+  const void* zero;
+  const void* bias;  // nullptr or [N]
+  void* Y;
+  int64_t M, N, K;
+  int x_dtype;
+  int meta_dtype;
+};
+cudaError_t launch_w4a16_gemm(const GemmJob& job, cudaStream_t stream);
+// Number of bounded waits inside the GEMM kernel that ran out of time since the library was
+// loaded (0 on every healthy run).
+cudaError_t read_gemm_timeouts(unsigned int* out);
+
 cudaError_t launch_quantize_meta(const void* meta, int dtype, int64_t n, int group, uint8_t* q,
                                  float* mm, cudaStream_t stream);
 cudaError_t launch_dequantize_meta(const uint8_t* q, const float* mm, int64_t n, int group,

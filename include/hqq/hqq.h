@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define HQQ_ABI_VERSION 2
+#define HQQ_ABI_VERSION 3
 
 typedef enum {
   HQQ_OK = 0,
@@ -253,6 +253,37 @@ hqq_status hqq_quantize_meta(const void* meta, hqq_dtype dtype, int64_t n, int g
 /* out_f32[i] = (q_u8[i] - zero2)*step2 of its run, in fp32. All pointers device. */
 hqq_status hqq_dequantize_meta(const void* q_u8, const void* mm, int64_t n, int group,
                                void* out_f32, cudaStream_t stream);
+
+/* The consumer of the packed format: the forward pass of an HQQ-quantized linear layer,
+ *     Y[m, n] = dtype( sum_k X[m, k] * W'[n, k]  (+ bias[n]) ),
+ * with W' the dequantized weight rounded once to the activation dtype exactly as
+ * hqq_dequantize writes it, W'[n, k] = dtype((float(Q[n, k]) - zero[g]) * scale[g]),
+ * g = n*(K/64) + k/64, and the sum accumulated in fp32 on the tensor cores ("HQQ
+ * calibration-free guide" (lnwmold.com) §3.2: a quantized layer computes in its compute
+ * dtype from the dequantized weight; §4.2: the axis=1 backends fuse the dequantization
+ * into the matrix product). The dequantized weight is never written to memory.
+ *   X          device, row-major [M, K] of x_dtype (HQQ_BF16 or HQQ_F16), 16-byte aligned.
+ *   Wq_packed, scale, zero
+ *              the outputs of hqq_quantize / hqq_quantize_ex for W of shape [N, K]
+ *              (rows = N output features, cols = K input features) with params->nbits 4,
+ *              group_size 64, axis 1 and no second level; scale and zero are
+ *              params->meta_dtype (F16, BF16 or F32). Wq_packed 16-byte aligned.
+ *   bias       NULL or device [N] of x_dtype.
+ *   Y          device, row-major [M, N] of x_dtype, 16-byte aligned; must not overlap the
+ *              inputs.
+ * Shapes: K % 64 == 0 and N % 8 == 0 (HQQ_ERR_SHAPE otherwise), M, N, K < 2^31. K == 0 gives
+ * Y = bias (or 0). Other nbits / group_size / axis, or quant_scale / quant_zero, return
+ * HQQ_ERR_UNSUPPORTED. The solver fields of params are ignored. */
+hqq_status hqq_linear(const void* X, int64_t M, int64_t K, hqq_dtype x_dtype,
+                      const void* Wq_packed, const void* scale, const void* zero,
+                      const void* bias, int64_t N, const hqq_params* params, void* Y,
+                      cudaStream_t stream);
+
+/* Kernels that wait on barriers inside a CTA (hqq_linear) bound each wait by about two
+ * seconds; a wait that runs out sets the CTA's outputs aside (not written), frees its
+ * resources and is counted. *count receives the number counted since the library was
+ * loaded on the current device (0 on every healthy run). Synchronises the device. */
+hqq_status hqq_wait_timeouts(unsigned int* count);
 
 /* Human-readable name of a status code (static storage). */
 const char* hqq_status_string(hqq_status status);

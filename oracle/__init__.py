@@ -193,3 +193,37 @@ def dequantize_meta(q, mm, group: int) -> np.ndarray:
     out = np.zeros(q.size, np.float32)
     _load().hqq_oracle_dequantize_meta(_ptr(q), _ptr(mm), q.size, group, _ptr(out))
     return out
+
+
+def round_to_dtype(a, dtype: str) -> np.ndarray:
+    """Round fp32 values once, to nearest with ties to even, to ``"bf16"`` or ``"f16"``;
+    returned as fp32 (which holds every such value exactly). ``"f32"`` returns a copy.
+
+    bf16 keeps the upper 16 bits of the fp32 pattern: adding 0x7FFF plus the lowest kept bit
+    and truncating rounds half to even (finite inputs; the path produces no NaN)."""
+    x = _f32(a)
+    if dtype == "f32":
+        return x.copy()
+    if dtype == "f16":
+        return x.astype(np.float16).astype(np.float32)
+    if dtype != "bf16":
+        raise ValueError(dtype)
+    b = x.view(np.uint32).astype(np.uint64)
+    r = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
+    return r.astype(np.uint32).view(np.float32).reshape(x.shape)
+
+
+def linear(X, codes, scale, zero, N: int, K: int, dtype: str, bias=None) -> np.ndarray:
+    """Forward pass of a quantized linear layer, in fp64: Y[m, n] = sum_k X[m, k]·W'[n, k]
+    (+ bias[n]), where W' is the axis-1, group-64 weight [N, K] dequantized by
+    ``dequantize`` and rounded once to the compute dtype ("HQQ calibration-free guide"
+    (lnwmold.com) §3.2: the layer dequantizes to compute_dtype and multiplies; §4.2: the
+    axis=1 backends fuse the two). X holds the activations' exact values (fp32 array of
+    bf16/fp16 numbers) [M, K]; codes are in g order. The product is numpy's float64 matmul:
+    a library primitive whose result differs from the exact sum by far less than any fp32
+    accumulation does. The caller rounds Y to the compute dtype where it compares bits."""
+    Wd = round_to_dtype(dequantize(codes, scale, zero, N, K, 64, 1), dtype)
+    Y = np.asarray(X, dtype=np.float64) @ Wd.astype(np.float64).T
+    if bias is not None:
+        Y = Y + np.asarray(bias, dtype=np.float64)[None, :]
+    return Y

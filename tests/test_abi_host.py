@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(L):
     assert "hqq_quantize" in names and "hqq_dequantize" in names and len(names) >= 12
     for n in names:
         assert hasattr(L, n), n
-    assert L.hqq_abi_version() == 2
+    assert L.hqq_abi_version() == 3
 
 
 def test_size_helpers_match_layout(L):
@@ -155,3 +155,35 @@ def test_unknown_flags_are_rejected(L):
                              0, None) == INVALID
     arr = (hqq.HQQMatrix * 1)(hqq.HQQMatrix(FAKE, 64, 128, FAKE, FAKE, FAKE))
     assert L.hqq_quantize_batched(arr, 1, ctypes.byref(p), None) == INVALID
+
+
+def test_linear_validates_before_launch(L):
+    BF16, F16, F32 = 1, 0, 2
+    good = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16)
+
+    def call(M=256, K=128, xdt=BF16, X=FAKE, W=FAKE, s=FAKE, z=FAKE, b=None, N=256,
+             prm=good, Y=FAKE):
+        return L.hqq_linear(X, M, K, xdt, W, s, z, b, N,
+                            ctypes.byref(prm) if prm is not None else None, Y, None)
+
+    assert call(prm=None) == INVALID
+    assert call(M=-1) == INVALID
+    assert call(xdt=F32) == UNSUPPORTED
+    for kw in ({"nbits": 3}, {"group_size": 32}, {"axis": 0}, {"quant_scale": True}):
+        args = dict(nbits=4, group_size=64, axis=1, w_dtype=torch.bfloat16)
+        args.update(kw)
+        assert call(prm=hqq.make_params(**args)) == UNSUPPORTED, kw
+    bad_meta = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16)
+    bad_meta.meta_dtype = 3
+    assert call(prm=bad_meta) == INVALID
+    assert call(K=96) == SHAPE
+    assert call(N=260) == SHAPE
+    assert call(M=1 << 31) == SHAPE
+    assert call(Y=None) == INVALID
+    assert call(X=None) == INVALID
+    assert call(X=FAKE_ODD) == ALIGN
+    assert call(Y=FAKE + 8) == ALIGN
+    assert call(b=FAKE + 1) == ALIGN
+    # nothing to do: valid arguments with M == 0 or N == 0 return at once, pointers unused
+    assert call(M=0, X=None, W=None, s=None, z=None, Y=None) == OK
+    assert call(N=0, X=None, W=None, s=None, z=None, Y=None) == OK

@@ -370,3 +370,72 @@ def test_deterministic_and_thread_count_invariant():
     b = oracle.quantize(W, 4, 64, 1, 20, **PARAMS, nthreads=4)
     for x, y in zip(a, b):
         assert np.array_equal(np.asarray(x).view(np.uint8), np.asarray(y).view(np.uint8))
+
+
+# ---------------------------------------------------------------- the quantized linear layer
+
+def test_round_to_bf16_ties_and_library():
+    # hand-derived: bf16 keeps 8 significant bits, so its spacing at 1 is 2^-7
+    x = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8), 1 + 2.0 ** -8 + 2.0 ** -20,
+                  2.0 ** -130], F32)
+    want = np.array([1.0, 1 + 2.0 ** -6, -1.0, 1 + 2.0 ** -7, 2.0 ** -130], F32)
+    assert np.array_equal(oracle.round_to_dtype(x, "bf16"), want)
+    # library routine: torch's fp32 -> bf16 conversion rounds to nearest even as well
+    import torch
+    r = (np.random.default_rng(5).standard_normal(200_000) * 37.0).astype(F32)
+    lib = torch.from_numpy(r).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(oracle.round_to_dtype(r, "bf16"), lib)
+    assert np.array_equal(oracle.round_to_dtype(r, "f16"), r.astype(np.float16).astype(F32))
+
+
+def _random_layer(N, K, seed, meta_scale=0.01):
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 16, size=N * K, dtype=np.uint8)
+    ng = N * K // 64
+    scale = oracle.round_to_dtype((rng.random(ng) * meta_scale + 1e-4).astype(F32), "bf16")
+    zero = oracle.round_to_dtype((rng.random(ng) * 15).astype(F32), "bf16")
+    return codes, scale, zero
+
+
+def test_linear_closed_form_constant_group():
+    # one group per row, every code c_n, scale s_n, zero z_n, X = all ones:
+    # Y[m, n] = 64·bf16((c_n - z_n)·s_n) exactly (64 equal terms, power-of-two multiple)
+    N, K = 8, 64
+    c = np.arange(N, dtype=np.uint8) * 2
+    codes = np.repeat(c, K)
+    scale = np.array([0.5, 0.25, 1.0, 2.0, 0.125, 0.75, 1.5, 3.0], F32)
+    zero = np.array([0.0, 1.0, 3.0, 7.5, 15.0, 2.25, 0.5, 8.0], F32)
+    X = np.ones((3, K), F32)
+    Y = oracle.linear(X, codes, scale, zero, N, K, "bf16")
+    want = 64.0 * ((c.astype(np.float64) - zero) * scale)  # every (c - z)·s is exact in bf16
+    assert np.array_equal(Y, np.broadcast_to(want, (3, N)))
+    bias = np.array([1, -2, 3, -4, 5, -6, 7, -8], F32)
+    assert np.array_equal(oracle.linear(X, codes, scale, zero, N, K, "bf16", bias) - Y,
+                          np.broadcast_to(bias.astype(np.float64), (3, N)))
+
+
+def test_linear_one_hot_rows_give_transposed_weight():
+    # X = identity: Y[k, n] = W'[n, k]. Fails on a transposed operand or a wrong group index.
+    N, K = 24, 192
+    codes, scale, zero = _random_layer(N, K, 3)
+    Y = oracle.linear(np.eye(K, dtype=F32), codes, scale, zero, N, K, "bf16")
+    Wd = np.empty((N, K), np.float64)
+    for n in range(N):  # element by element from the definition
+        for k in range(K):
+            g = n * (K // 64) + k // 64
+            v = F32(F32(F32(codes[n * K + k]) - zero[g]) * scale[g])
+            Wd[n, k] = oracle.round_to_dtype(np.array([v], F32), "bf16")[0]
+    assert np.array_equal(Y, Wd.T)
+
+
+def test_linear_matches_brute_force_sum():
+    N, K, M = 16, 128, 5
+    codes, scale, zero = _random_layer(N, K, 4)
+    rng = np.random.default_rng(6)
+    X = oracle.round_to_dtype(rng.standard_normal((M, K)).astype(F32), "bf16")
+    Y = oracle.linear(X, codes, scale, zero, N, K, "bf16")
+    Wd = oracle.round_to_dtype(oracle.dequantize(codes, scale, zero, N, K, 64, 1), "bf16")
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(X[m, k])) * Fraction(float(Wd[n, k])) for k in range(K))
+            assert abs(Fraction(Y[m, n]) - exact) <= Fraction(1, 2 ** 40) * (1 + abs(exact))
