@@ -403,7 +403,7 @@ HQQ_EXPORT hqq_status hqq_linear(const void* X, int64_t M, int64_t K, hqq_dtype 
   if (!wdtype_ok(prm.meta_dtype)) return HQQ_ERR_INVALID_ARG;
   if (K % 64 != 0 || N % 8 != 0) return HQQ_ERR_SHAPE;
   if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) ||
-      (M + 255) / 256 > 65535)
+      (N + 255) / 256 > 65535)
     return HQQ_ERR_SHAPE;
   if (M == 0 || N == 0) return HQQ_OK;
   if (!Y) return HQQ_ERR_INVALID_ARG;

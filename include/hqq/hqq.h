@@ -271,7 +271,8 @@ hqq_status hqq_dequantize_meta(const void* q_u8, const void* mm, int64_t n, int 
  *   bias       NULL or device [N] of x_dtype.
  *   Y          device, row-major [M, N] of x_dtype, 16-byte aligned; must not overlap the
  *              inputs.
- * Shapes: K % 64 == 0 and N % 8 == 0 (HQQ_ERR_SHAPE otherwise), M, N, K < 2^31. K == 0 gives
+ * Shapes: K % 64 == 0 and N % 8 == 0 (HQQ_ERR_SHAPE otherwise), M, K < 2^31, N <= 65535*256.
+ * K == 0 gives
  * Y = bias (or 0). Other nbits / group_size / axis, or quant_scale / quant_zero, return
  * HQQ_ERR_UNSUPPORTED. The solver fields of params are ignored. */
 hqq_status hqq_linear(const void* X, int64_t M, int64_t K, hqq_dtype x_dtype,
