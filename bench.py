@@ -270,6 +270,10 @@ def run_ours(args, rank, world, dev):
         res["e2e"] = run_e2e(hqq, wl, Ws, outs, dev, args)
     if rank == 0 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(wl, Ws, args.cpu_seconds)
+    if rank == 0 and not args.no_linear:
+        del Ws, outs, deqs, qbatch, dbatch
+        torch.cuda.empty_cache()
+        res["w4a16_linear"] = run_linear(hqq, dev, args)
     return res
 
 
@@ -323,6 +327,104 @@ def _traffic_per_launch(avg_weights):
     if t.get("solver_source_sha1") != solver_source_digest():
         return None
     return round(t["dram_bytes_per_weight"] * avg_weights)
+
+
+def linear_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("hqq_gemm.cu", "hqq_device.cuh"):
+        with open(os.path.join(HERE, "calibration_free_weight_hqq_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def run_linear(hqq, dev, args, tokens: int = 4096):
+    """The consumer of the packed format (row f2): the seven linear layers of one Llama-7B
+    block (q, k, v, o [4096,4096]; gate, up [11008,4096]; down [4096,11008]) quantized to
+    4-bit g64 axis 1, applied to a prefill batch of `tokens` bf16 tokens with hqq_linear
+    (dequantization fused into the tcgen05 GEMM, bit-identical to hqq_dequantize). Beside it,
+    in the same run: the unfused path (hqq_dequantize + torch.matmul on the bf16 result) and
+    cuBLAS on an already dequantized bf16 weight. L2 is flushed (256 MB write) before every
+    step; each launch is timed with CUDA events on the launching stream."""
+    from calibration_free_weight_hqq_b200 import synthetic, workloads
+    wl = workloads.llama7b_block_4b()
+    stream = torch.cuda.current_stream()
+    layers = []
+    for m in wl.matrices:
+        W = workloads.make_weight(m, dev)
+        pk, sc, zr = hqq.hqq_quantize(W, 4, 64, 1)
+        X = synthetic.activations(tokens, m.cols, seed=m.seed + 7, device=dev)
+        Y = torch.empty(tokens, m.rows, dtype=torch.bfloat16, device=dev)
+        Wd = hqq.hqq_dequantize(pk, sc, zr, m.rows, m.cols, 4, 64, 1)
+        layers.append((m, X, pk, sc, zr, Y, Wd))
+        del W
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    scratch = torch.empty(max(m.rows * m.cols for m, *_ in layers), dtype=torch.bfloat16,
+                          device=dev)  # the unfused path's dequantized weight
+    flops = sum(2.0 * tokens * m.rows * m.cols for m, *_ in layers)
+
+    def timed(fn, steps):
+        per = []
+        for _ in range(args.warmup):
+            for L in layers:
+                fn(*L)
+        torch.cuda.synchronize()
+        for _ in range(steps):
+            flush.fill_(1)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in layers]
+            for (a, b), L in zip(evs, layers):
+                a.record(stream)
+                fn(*L)
+                b.record(stream)
+            torch.cuda.synchronize()
+            per.append(sum(a.elapsed_time(b) for a, b in evs))
+        return statistics.median(per)
+
+    ms_fused = timed(lambda m, X, pk, sc, zr, Y, Wd: hqq.hqq_linear(X, pk, sc, zr, m.rows, Y=Y,
+                                                                     stream=stream), args.steps)
+    ms_unfused = timed(lambda m, X, pk, sc, zr, Y, Wd: torch.matmul(
+        X, hqq.hqq_dequantize(pk, sc, zr, m.rows, m.cols, 4, 64, 1, stream=stream,
+                              out=scratch[:m.rows * m.cols].view(m.rows, m.cols)).t(), out=Y),
+        args.steps)
+    ms_cublas = timed(lambda m, X, pk, sc, zr, Y, Wd: torch.matmul(X, Wd.t(), out=Y), args.steps)
+    tf = flops / (ms_fused * 1e-3) / 1e12
+    peak, source = None, "fallback"
+    path = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            peak = json.load(f).get("bf16_tflops")
+        source = "measured"
+    if peak is None:
+        peak = 1590.0
+    # DRAM traffic of one 4096^3 launch from the committed ncu capture (the launches here
+    # have three shapes, so it is reported for that case, not scaled)
+    profiled = None
+    tpath = os.path.join(HERE, "profiles", "w4a16_gemm_kernel_traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            t = json.load(f)
+        if t.get("source_sha1") == linear_source_digest():
+            profiled = {"shape_MNK": [4096, 4096, 4096],
+                        "dram_bytes": t.get("dram_bytes_per_launch_4096x4096x4096"),
+                        "algorithmic_bytes": 2 * 4096 * 4096 * 2 + 4096 * 4096 // 2 + 4096 * 64 * 4}
+    return {
+        "metric": "fused 4-bit linear TFLOP/s", "value": round(tf, 1), "unit": "TFLOP/s",
+        "workload": f"Llama-7B block linear layers, {tokens} tokens, bf16 activations, "
+                    "4-bit g64 axis-1 weights",
+        "ms_per_step": round(ms_fused, 4), "launches_per_step": len(layers),
+        "unfused_dequantize_plus_cublas_tflops": round(flops / (ms_unfused * 1e-3) / 1e12, 1),
+        "cublas_bf16_weight_tflops": round(flops / (ms_cublas * 1e-3) / 1e12, 1),
+        "roofline": {"bound": "tensor", "kernel": "w4a16_gemm_2sm_kernel (tcgen05 cta_group::2)",
+                     "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(tf / peak, 4), "traffic": None,
+                     "traffic_profiled_case": profiled,
+                     "algorithmic": "2*M*N*K flops per launch",
+                     "peak_source": f"bf16 dense, {source} (burst: the kernel is timed alone)"},
+        "l2": "flushed before every step",
+        "wait_timeouts": hqq.hqq_wait_timeouts(),
+        "gpu_launches": len(layers) * args.steps,
+    }
 
 
 def run_e2e(hqq, wl, Ws, outs, dev, args):
@@ -512,6 +614,30 @@ def probe_hbm(gib: float = 1.0):
     return res
 
 
+def single_linear(reps: int = 10):
+    """One 4096 x 4096 x 4096 hqq_linear launch (bf16, 4-bit g64): the ncu profiling case."""
+    import calibration_free_weight_hqq_b200 as hqq
+    from calibration_free_weight_hqq_b200 import synthetic
+    M = N = K = 4096
+    W = synthetic.weight(N, K, seed=11, dtype=torch.bfloat16, device="cuda")
+    pk, s, z = hqq.hqq_quantize(W, 4, 64, 1)
+    X = synthetic.activations(M, K, seed=12, device="cuda")
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    for _ in range(2):
+        hqq.hqq_linear(X, pk, s, z, N, Y=Y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        hqq.hqq_linear(X, pk, s, z, N, Y=Y)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    return {"single": "linear", "shape": [M, N, K], "ms": round(ms, 4),
+            "TFLOP_per_s": round(2.0 * M * N * K / ms / 1e9, 1),
+            "wait_timeouts": hqq.hqq_wait_timeouts()}
+
+
 def single(kind: str, reps: int = 10):
     """One [16384, 8192] bf16 matrix (134M weights, 268 MB: larger than L2), 4-bit g64:
     time `reps` solver or dequantize launches after warm-up (the small case the ncu
@@ -554,13 +680,16 @@ def main():
     ap.add_argument("--per-matrix", action="store_true",
                     help="one launch per matrix instead of the batched whole-model calls")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-linear", action="store_true",
+                    help="skip the fused 4-bit linear-layer measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--probe-sfu", action="store_true",
                     help="measure the lg2/ex2 issue rate behind the roofline peak and exit")
     ap.add_argument("--probe-hbm", action="store_true",
                     help="measure HBM read-only, write-only and copy bandwidth and exit")
-    ap.add_argument("--single", choices=["quantize", "dequantize"],
-                    help="time one [16384,8192] matrix (the profiling case) and exit")
+    ap.add_argument("--single", choices=["quantize", "dequantize", "linear"],
+                    help="time one [16384,8192] matrix, or one 4096^3 linear layer (the "
+                         "profiling cases), and exit")
     args = ap.parse_args()
     if args.probe_sfu:
         print(json.dumps(probe_sfu()), flush=True)
@@ -569,7 +698,8 @@ def main():
         print(json.dumps(probe_hbm()), flush=True)
         return
     if args.single:
-        print(json.dumps(single(args.single)), flush=True)
+        print(json.dumps(single_linear() if args.single == "linear" else single(args.single)),
+              flush=True)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

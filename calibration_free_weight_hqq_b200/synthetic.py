@@ -49,3 +49,13 @@ def weight(rows: int, cols: int, *, seed: int, dtype=torch.bfloat16, outlier_rat
         W = torch.where(mask, W * mag, W)
         del mag, mask
     return W.to(dtype)
+
+
+def activations(rows: int, cols: int, *, seed: int, dtype=torch.bfloat16,
+                device="cpu") -> torch.Tensor:
+    """Seeded layer inputs for the quantized linear layer: X[m, k] ~ N(0, 1), rounded once
+    to dtype (stands in for a prefill batch of `rows` tokens; normalised hidden states of a
+    Llama block have unit scale)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return torch.randn(rows, cols, generator=g, device=device, dtype=torch.float32).to(dtype)
