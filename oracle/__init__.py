@@ -227,3 +227,62 @@ def linear(X, codes, scale, zero, N: int, K: int, dtype: str, bias=None) -> np.n
     if bias is not None:
         Y = Y + np.asarray(bias, dtype=np.float64)[None, :]
     return Y
+
+
+def _mx_sigs(L):
+    u8p = ctypes.c_void_p
+    L.hqq_oracle_e2m1_encode.argtypes = [ctypes.c_float]
+    L.hqq_oracle_e2m1_encode.restype = ctypes.c_uint8
+    L.hqq_oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+    L.hqq_oracle_e2m1_decode.restype = ctypes.c_float
+    L.hqq_oracle_mx_exponent.argtypes = [u8p, ctypes.c_int]
+    L.hqq_oracle_mx_exponent.restype = ctypes.c_int
+    L.hqq_oracle_mxfp4_quantize.argtypes = [u8p, ctypes.c_int64, ctypes.c_int64, u8p, u8p]
+    L.hqq_oracle_mxfp4_dequantize.argtypes = [u8p, u8p, ctypes.c_int64, ctypes.c_int64, u8p]
+
+
+def e2m1_encode(v: float) -> int:
+    """One FP4 E2M1 code (sign bit 3, magnitude index 0..7) for an fp32 value: nearest
+    E2M1 value, ties to the even mantissa bit, saturating at 6 (MX conversion)."""
+    L = _load()
+    _mx_sigs(L)
+    return int(L.hqq_oracle_e2m1_encode(float(np.float32(v))))
+
+
+def e2m1_decode(code: int) -> float:
+    L = _load()
+    _mx_sigs(L)
+    return float(L.hqq_oracle_e2m1_decode(code))
+
+
+def mx_exponent(v) -> int:
+    """Shared exponent of one block: floor(log2 max|v|) - 2, clamped to [-127, 127]."""
+    L = _load()
+    _mx_sigs(L)
+    a = _f32(v).ravel()
+    return int(L.hqq_oracle_mx_exponent(_ptr(a), a.size))
+
+
+def mxfp4_quantize(W):
+    """MXFP4 encoding of the fp32 matrix W [rows, cols] (cols % 32 == 0), blocks of 32 along
+    rows: returns (codes uint8 [rows*cols/2], scales uint8 [rows*cols/32] = e + 127)."""
+    L = _load()
+    _mx_sigs(L)
+    W = _f32(W)
+    rows, cols = W.shape
+    assert cols % 32 == 0
+    codes = np.zeros(rows * cols // 2, np.uint8)
+    scales = np.zeros(rows * cols // 32, np.uint8)
+    L.hqq_oracle_mxfp4_quantize(_ptr(W), rows, cols, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def mxfp4_dequantize(codes, scales, rows: int, cols: int) -> np.ndarray:
+    """fp32 [rows, cols]: E2M1 value x 2^(scale - 127)."""
+    L = _load()
+    _mx_sigs(L)
+    c = np.ascontiguousarray(np.asarray(codes, np.uint8).ravel())
+    s = np.ascontiguousarray(np.asarray(scales, np.uint8).ravel())
+    out = np.zeros((rows, cols), np.float32)
+    L.hqq_oracle_mxfp4_dequantize(_ptr(c), _ptr(s), rows, cols, _ptr(out))
+    return out

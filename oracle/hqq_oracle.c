@@ -376,3 +376,77 @@ void hqq_oracle_dequantize_meta(const uint8_t* q, const float* mm, int64_t n, in
     out[k] = d * mm[2 * i];
   }
 }
+
+/* ------------------------------------------------------------------ MXFP4 weight-only
+ * [guide 5.1] "HQQ calibration-free guide" (lnwmold.com) §5.1 lists an mxfp4 weight-only
+ * mode among the on-the-fly quantization modes; the pages give no further definition, so
+ * the encoding is the plainest reading: the Open Compute Project Microscaling (MX) format
+ * MXFP4 - blocks of 32 consecutive elements along a row share one E8M0 scale (a power of
+ * two, stored as the biased exponent e + 127), and every element is an FP4 E2M1 number
+ * (sign, 2 exponent bits, 1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6).
+ * Conversion as that specification defines it:
+ *   e  = floor(log2(max_i |V_i|)) - 2      (2 = exponent of E2M1's largest normal 6 = 1.5*2^2)
+ *        clamped to the E8M0 range [-127, 127]; an all-zero block takes e = -127 (reading R14)
+ *   P_i = V_i / 2^e rounded to the nearest E2M1 value, ties to the value with an even
+ *        mantissa bit, magnitudes above 6 saturating to 6; the sign is kept (reading R15:
+ *        -0 encodes as sign bit set, magnitude 0)
+ *   dequantization: V'_i = P_i * 2^e.
+ * Codes are packed two per byte, element 2j in the low nibble (as the 4-bit integer codes). */
+static const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+uint8_t hqq_oracle_e2m1_encode(float v) {
+  const uint8_t sign = signbit(v) ? 8 : 0;
+  const float a = fabsf(v);
+  int best = 0;
+  for (int m = 1; m < 8; ++m) {  /* nearest grid value; on a tie the even mantissa bit */
+    const float db = fabsf(a - kE2M1[best]), dm = fabsf(a - kE2M1[m]);
+    if (dm < db || (dm == db && (m & 1) == 0)) best = m;
+  }
+  if (a > 6.0f) best = 7; /* saturation (also covered by the search above) */
+  return (uint8_t)(sign | best);
+}
+
+float hqq_oracle_e2m1_decode(uint8_t code) {
+  const float m = kE2M1[code & 7];
+  return (code & 8) ? -m : m;
+}
+
+int hqq_oracle_mx_exponent(const float* v, int n) {
+  float amax = 0.0f;
+  for (int i = 0; i < n; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  if (amax == 0.0f) return -127;
+  int ex;
+  (void)frexpf(amax, &ex); /* amax = f * 2^ex, f in [0.5, 1): floor(log2 amax) = ex - 1 */
+  int e = (ex - 1) - 2;
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return e;
+}
+
+void hqq_oracle_mxfp4_quantize(const float* W, int64_t rows, int64_t cols, uint8_t* codes,
+                               uint8_t* scales) {
+  const int64_t nb = rows * cols / 32;
+  for (int64_t b = 0; b < nb; ++b) {
+    const float* v = W + b * 32; /* row-major: block b = (r, c/32) */
+    const int e = hqq_oracle_mx_exponent(v, 32);
+    scales[b] = (uint8_t)(e + 127);
+    for (int i = 0; i < 32; ++i) {
+      const float x = ldexpf(v[i], -e); /* exact division by the power of two */
+      const uint8_t c = hqq_oracle_e2m1_encode(x);
+      const int64_t k = b * 32 + i;
+      if ((k & 1) == 0)
+        codes[k / 2] = c;
+      else
+        codes[k / 2] |= (uint8_t)(c << 4);
+    }
+  }
+}
+
+void hqq_oracle_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows,
+                                 int64_t cols, float* out) {
+  const int64_t n = rows * cols;
+  for (int64_t k = 0; k < n; ++k) {
+    const uint8_t c = (k & 1) ? (uint8_t)(codes[k / 2] >> 4) : (uint8_t)(codes[k / 2] & 15);
+    out[k] = ldexpf(hqq_oracle_e2m1_decode(c), (int)scales[k / 32] - 127);
+  }
+}

@@ -439,3 +439,84 @@ def test_linear_matches_brute_force_sum():
         for n in range(N):
             exact = sum(Fraction(float(X[m, k])) * Fraction(float(Wd[n, k])) for k in range(K))
             assert abs(Fraction(Y[m, n]) - exact) <= Fraction(1, 2 ** 40) * (1 + abs(exact))
+
+
+# ---------------------------------------------------------------- MXFP4 (row f3)
+
+def _e2m1_from_fields(code):
+    """E2M1 from its bit fields (sign | 2 exponent bits | 1 mantissa bit, bias 1): exponent
+    field 0 is subnormal (value = M/2), otherwise 2^(E-1) * (1 + M/2)."""
+    s = -1.0 if code & 8 else 1.0
+    E, M = (code >> 1) & 3, code & 1
+    return s * (M * 0.5 if E == 0 else 2.0 ** (E - 1) * (1 + M / 2))
+
+
+def test_e2m1_decode_matches_bit_fields():
+    for c in range(16):
+        assert oracle.e2m1_decode(c) == _e2m1_from_fields(c), c
+    # the largest normal is 1.5 * 2^2 = 6, the exponent the MX scale rule subtracts
+    assert max(_e2m1_from_fields(c) for c in range(16)) == 6.0
+
+
+def test_e2m1_encode_is_nearest_ties_to_even_with_saturation():
+    grid = np.array([_e2m1_from_fields(c) for c in range(8)])
+    mids = (grid[1:] + grid[:-1]) / 2
+    xs = np.concatenate([grid, mids, mids + 1e-3, mids - 1e-3, [6.5, 7.9, 8.0, 1e6],
+                         np.linspace(0, 7, 701)])
+    for x in xs:
+        for sgn in (1.0, -1.0):
+            v = np.float32(sgn * x)
+            code = oracle.e2m1_encode(v)
+            a = min(abs(float(v)), 6.0)  # saturation: anything above 6 becomes 6
+            d = np.abs(grid - a)
+            cands = np.flatnonzero(d == d.min())
+            want = cands[0] if len(cands) == 1 else [c for c in cands if c % 2 == 0][0]
+            assert code & 7 == want, (v, code)
+            assert (code >> 3) == (1 if np.signbit(v) else 0)
+
+
+def test_mx_exponent_closed_form():
+    rng = np.random.default_rng(14)
+    for _ in range(300):
+        v = (rng.standard_normal(32) * 10.0 ** rng.uniform(-6, 6)).astype(F32)
+        amax = float(np.max(np.abs(v)))
+        want = int(np.floor(np.log2(amax))) - 2
+        assert oracle.mx_exponent(v) == max(-127, min(127, want))
+    assert oracle.mx_exponent([4.0]) == 0 and oracle.mx_exponent([3.999]) == -1
+    assert oracle.mx_exponent([-8.0, 1.0]) == 1
+    assert oracle.mx_exponent(np.zeros(32, F32)) == -127
+
+
+def test_mxfp4_exact_blocks_round_trip_and_packing():
+    rng = np.random.default_rng(15)
+    rows, cols = 6, 96
+    W = np.zeros((rows, cols), F32)
+    for b in range(rows * cols // 32):
+        e = int(rng.integers(-20, 20))
+        vals = np.array([_e2m1_from_fields(int(c)) for c in rng.integers(0, 16, 32)])
+        vals[0] = 6.0 if b % 2 else -4.0  # the block maximum fixes the exponent at e
+        W.reshape(-1)[b * 32:(b + 1) * 32] = (vals * 2.0 ** e).astype(F32)
+    codes, scales = oracle.mxfp4_quantize(W)
+    back = oracle.mxfp4_dequantize(codes, scales, rows, cols)
+    nz = W != 0
+    assert np.array_equal(back[nz], W[nz]) and np.all(back[~nz] == 0)
+    # two codes per byte, element 2j in the low nibble: the 4-bit integer packing
+    flat = np.array([oracle.e2m1_encode(np.float32(x) / np.float32(2.0 ** (int(s) - 127)))
+                     for x, s in zip(W.reshape(-1), np.repeat(scales, 32))], np.uint8)
+    assert np.array_equal(codes, oracle.pack(flat, 4))
+
+
+def test_mxfp4_error_bound_and_extremes():
+    rng = np.random.default_rng(16)
+    W = (rng.standard_normal((64, 256)) * np.exp(rng.standard_normal((64, 1)))).astype(F32)
+    codes, scales = oracle.mxfp4_quantize(W)
+    back = oracle.mxfp4_dequantize(codes, scales, 64, 256)
+    X = 2.0 ** (np.repeat(scales.astype(np.int64) - 127, 32).reshape(64, 256))
+    x = np.abs(W) / X  # scaled magnitudes lie in [0, 8)
+    assert x.max() < 8
+    half_gap = np.where(x <= 2, 0.25, np.where(x <= 4, 0.5, 1.0))
+    bound = np.where(x <= 6, half_gap, x - 6) * X
+    assert np.all(np.abs(W - back) <= bound * (1 + 1e-6))
+    # every block's largest magnitude lands on 4 or 6 (scaled max in [4, 8))
+    top = np.abs(back).reshape(-1, 32).max(1) / X.reshape(-1, 32)[:, 0]
+    assert np.all((top == 4) | (top == 6))
