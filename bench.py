@@ -274,6 +274,7 @@ def run_ours(args, rank, world, dev):
         del Ws, outs, deqs, qbatch, dbatch
         torch.cuda.empty_cache()
         res["w4a16_linear"] = run_linear(hqq, dev, args)
+        res["mxfp4_weightonly"] = run_mxfp4(hqq, dev, args)
     return res
 
 
@@ -425,6 +426,49 @@ def run_linear(hqq, dev, args, tokens: int = 4096):
         "wait_timeouts": hqq.hqq_wait_timeouts(),
         "gpu_launches": len(layers) * args.steps,
     }
+
+
+def run_mxfp4(hqq, dev, args):
+    """Row f3, the MXFP4 weight-only encoding: one [28672, 8192] bf16 weight (the 70B-class
+    MLP shape, 235M weights, 470 MB: above L2), encode and decode timed separately with CUDA
+    events over `steps` launches after warm-up. Both are HBM-bound: 2.53125 algorithmic bytes
+    per weight (read 2 B bf16; write 0.5 B codes + 1/32 B scale, or the reverse)."""
+    from calibration_free_weight_hqq_b200 import synthetic
+    rows, cols = 28672, 8192
+    W = synthetic.weight(rows, cols, seed=3, dtype=torch.bfloat16, device=dev)
+    codes, scales = hqq.hqq_mxfp4_quantize(W)
+    D = torch.empty_like(W)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    ms_q = timed(lambda: hqq.hqq_mxfp4_quantize(W, codes=codes, scales=scales))
+    ms_d = timed(lambda: hqq.hqq_mxfp4_dequantize(codes, scales, rows, cols, out=D))
+    n = rows * cols
+    bpw = 2.53125
+    hbm = peaks()["hbm_gbs"]
+    gbs_q, gbs_d = n * bpw / (ms_q * 1e-3) / 1e9, n * bpw / (ms_d * 1e-3) / 1e9
+    return {"metric": "MXFP4 weight-only encode Gweights/s", "unit": "Gweights/s",
+            "value": round(n / (ms_q * 1e-3) / 1e9, 1),
+            "decode_Gweights_per_s": round(n / (ms_d * 1e-3) / 1e9, 1),
+            "workload": "one [28672, 8192] bf16 weight, blocks of 32 along rows",
+            "ms_encode": round(ms_q, 4), "ms_decode": round(ms_d, 4),
+            "roofline": {"bound": "hbm", "kernel": "mxfp4_quantize_kernel",
+                         "achieved": round(gbs_q, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs_q / hbm, 4), "traffic": None,
+                         "algorithmic": "2.53125 B/weight x 234881024 weights",
+                         "decode_achieved": round(gbs_d, 1),
+                         "decode_frac": round(gbs_d / hbm, 4)},
+            "gpu_launches": 2 * args.steps}
 
 
 def run_e2e(hqq, wl, Ws, outs, dev, args):

@@ -102,10 +102,12 @@ def lib() -> ctypes.CDLL:
             L.hqq_linear.argtypes = [P, i64, i64, i32, P, P, P, P, i64,
                                      ctypes.POINTER(HQQParams), P, P]
             L.hqq_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+            L.hqq_mxfp4_quantize.argtypes = [P, i32, i64, i64, P, P, P]
+            L.hqq_mxfp4_dequantize.argtypes = [P, P, i64, i64, i32, P, P]
             for f in ("hqq_quantize", "hqq_dequantize", "hqq_quantize_ex", "hqq_dequantize_ex",
                       "hqq_quantize_meta", "hqq_dequantize_meta", "hqq_quantize_ex_noalloc",
                       "hqq_quantize_batched", "hqq_dequantize_batched", "hqq_linear",
-                      "hqq_wait_timeouts"):
+                      "hqq_wait_timeouts", "hqq_mxfp4_quantize", "hqq_mxfp4_dequantize"):
                 getattr(L, f).restype = i32
             L.hqq_packed_bytes.argtypes = [i64, i64, i32, i32, i32]
             L.hqq_packed_bytes.restype = sz
@@ -399,3 +401,34 @@ def hqq_wait_timeouts() -> int:
     n = ctypes.c_uint(0)
     _check(lib().hqq_wait_timeouts(ctypes.byref(n)), "hqq_wait_timeouts")
     return int(n.value)
+
+
+def hqq_mxfp4_quantize(W: torch.Tensor, *, codes: Optional[torch.Tensor] = None,
+                       scales: Optional[torch.Tensor] = None, stream=None):
+    """MXFP4 encoding of a 2-D CUDA weight (fp16/bf16/fp32, cols % 32 == 0): returns
+    (codes uint8 [rows, cols/2], scales uint8 [rows, cols/32] = e + 127)."""
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D")
+    rows, cols = W.shape
+    if codes is None:
+        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=W.device)
+    if scales is None:
+        scales = torch.empty(rows, cols // 32, dtype=torch.uint8, device=W.device)
+    st = lib().hqq_mxfp4_quantize(_cuda(W, "W"), _TORCH_DT.get(W.dtype, -1), rows, cols,
+                                  _cuda(codes, "codes"), _cuda(scales, "scales"),
+                                  _stream(stream))
+    _check(st, "hqq_mxfp4_quantize")
+    return codes, scales
+
+
+def hqq_mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, rows: int, cols: int,
+                         out_dtype=torch.bfloat16, *, out: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """Decode MXFP4 codes and scales to a [rows, cols] CUDA tensor of out_dtype."""
+    if out is None:
+        out = torch.empty(rows, cols, dtype=out_dtype, device=codes.device)
+    st = lib().hqq_mxfp4_dequantize(_cuda(codes, "codes"), _cuda(scales, "scales"), rows, cols,
+                                    _TORCH_DT.get(out.dtype, -1), _cuda(out, "out"),
+                                    _stream(stream))
+    _check(st, "hqq_mxfp4_dequantize")
+    return out

@@ -19,7 +19,7 @@ BUILD_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libhqq_b200.so")
 PROBE_LIB = os.path.join(HERE, "libhqq_probe.so")  # SFU throughput probe used by bench.py
 SOURCES = ["hqq_abi.cu", "hqq_quantize.cu", "hqq_quantize_stop.cu", "hqq_dequantize.cu",
-           "hqq_noalloc.cu", "hqq_gemm.cu"]
+           "hqq_noalloc.cu", "hqq_gemm.cu", "hqq_mx.cu"]
 HEADERS = ["hqq_device.cuh", "hqq_kernels.h", "hqq_quantize_impl.cuh"]
 PUBLIC_HEADER = os.path.join(ROOT, "include", "hqq", "hqq.h")
 

@@ -432,3 +432,38 @@ HQQ_EXPORT hqq_status hqq_wait_timeouts(unsigned int* count) {
   if (!count) return HQQ_ERR_INVALID_ARG;
   return cuda_status(hqqk::read_gemm_timeouts(count));
 }
+
+static hqq_status check_mx_shape(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return HQQ_ERR_INVALID_ARG;
+  if (cols % 32 != 0) return HQQ_ERR_SHAPE;
+  if (rows > 0 && cols > 0 && rows > kMaxElems / cols) return HQQ_ERR_SHAPE;
+  return HQQ_OK;
+}
+
+HQQ_EXPORT hqq_status hqq_mxfp4_quantize(const void* W, hqq_dtype dtype, int64_t rows,
+                                         int64_t cols, void* codes, void* scales,
+                                         cudaStream_t stream) {
+  hqq_status st = check_mx_shape(rows, cols);
+  if (st != HQQ_OK) return st;
+  if (!wdtype_ok(dtype)) return HQQ_ERR_UNSUPPORTED;
+  if (rows * cols == 0) return HQQ_OK;
+  if (!W || !codes || !scales) return HQQ_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(codes, 4)) return HQQ_ERR_ALIGNMENT;
+  return cuda_status(hqqk::launch_mxfp4_quantize(W, dtype, rows * cols,
+                                                 reinterpret_cast<uint8_t*>(codes),
+                                                 reinterpret_cast<uint8_t*>(scales), stream));
+}
+
+HQQ_EXPORT hqq_status hqq_mxfp4_dequantize(const void* codes, const void* scales, int64_t rows,
+                                           int64_t cols, hqq_dtype out_dtype, void* W_out,
+                                           cudaStream_t stream) {
+  hqq_status st = check_mx_shape(rows, cols);
+  if (st != HQQ_OK) return st;
+  if (!wdtype_ok(out_dtype)) return HQQ_ERR_UNSUPPORTED;
+  if (rows * cols == 0) return HQQ_OK;
+  if (!codes || !scales || !W_out) return HQQ_ERR_INVALID_ARG;
+  if (!aligned(codes, 4) || !aligned(W_out, 16)) return HQQ_ERR_ALIGNMENT;
+  return cuda_status(hqqk::launch_mxfp4_dequantize(reinterpret_cast<const uint8_t*>(codes),
+                                                   reinterpret_cast<const uint8_t*>(scales),
+                                                   rows * cols, out_dtype, W_out, stream));
+}

@@ -68,6 +68,12 @@ cudaError_t launch_w4a16_gemm(const GemmJob& job, cudaStream_t stream);
 // loaded (0 on every healthy run).
 cudaError_t read_gemm_timeouts(unsigned int* out);
 
+// MXFP4: n = rows*cols elements (n % 32 == 0), blocks of 32 consecutive elements.
+cudaError_t launch_mxfp4_quantize(const void* W, int dtype, int64_t n, uint8_t* codes,
+                                  uint8_t* scales, cudaStream_t stream);
+cudaError_t launch_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t n,
+                                    int out_dtype, void* out, cudaStream_t stream);
+
 cudaError_t launch_quantize_meta(const void* meta, int dtype, int64_t n, int group, uint8_t* q,
                                  float* mm, cudaStream_t stream);
 cudaError_t launch_dequantize_meta(const uint8_t* q, const float* mm, int64_t n, int group,

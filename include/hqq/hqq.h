@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define HQQ_ABI_VERSION 3
+#define HQQ_ABI_VERSION 4
 
 typedef enum {
   HQQ_OK = 0,
@@ -279,6 +279,25 @@ hqq_status hqq_linear(const void* X, int64_t M, int64_t K, hqq_dtype x_dtype,
                       const void* Wq_packed, const void* scale, const void* zero,
                       const void* bias, int64_t N, const hqq_params* params, void* Y,
                       cudaStream_t stream);
+
+/* MXFP4 weight-only encoding ("HQQ calibration-free guide" (lnwmold.com) §5.1 lists an
+ * mxfp4 weight-only mode; the encoding is the Open Compute Project Microscaling format
+ * MXFP4). W: device, row-major [rows, cols] of dtype (F16, BF16 or F32), 16-byte aligned,
+ * finite values; cols % 32 == 0 (HQQ_ERR_SHAPE otherwise). Blocks of 32 consecutive elements
+ * of a row share one scale 2^e, e = floor(log2(max |v|)) - 2 clamped to [-127, 127] (an
+ * all-zero block takes -127), written as the byte e + 127 to scales[block] (block = r*cols/32
+ * + c/32; rows*cols/32 bytes). Each element is v / 2^e rounded to the nearest FP4 E2M1 value
+ * (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6; ties to the even mantissa bit; above 6 saturates to
+ * 6; sign kept), as a 4-bit code sign<<3 | magnitude index, two per byte with element 2j in
+ * the low nibble (codes: rows*cols/2 bytes, 4-byte aligned). */
+hqq_status hqq_mxfp4_quantize(const void* W, hqq_dtype dtype, int64_t rows, int64_t cols,
+                              void* codes, void* scales, cudaStream_t stream);
+
+/* W_out[k] = E2M1 value of code k * 2^(scales[k/32] - 127), computed exactly and rounded once
+ * to out_dtype (F16, BF16 or F32); W_out: device [rows, cols], 16-byte aligned. */
+hqq_status hqq_mxfp4_dequantize(const void* codes, const void* scales, int64_t rows,
+                                int64_t cols, hqq_dtype out_dtype, void* W_out,
+                                cudaStream_t stream);
 
 /* Kernels that wait on barriers inside a CTA (hqq_linear) bound each wait by about two
  * seconds; a wait that runs out sets the CTA's outputs aside (not written), frees its

@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(L):
     assert "hqq_quantize" in names and "hqq_dequantize" in names and len(names) >= 12
     for n in names:
         assert hasattr(L, n), n
-    assert L.hqq_abi_version() == 3
+    assert L.hqq_abi_version() == 4
 
 
 def test_size_helpers_match_layout(L):
@@ -187,3 +187,17 @@ def test_linear_validates_before_launch(L):
     # nothing to do: valid arguments with M == 0 or N == 0 return at once, pointers unused
     assert call(M=0, X=None, W=None, s=None, z=None, Y=None) == OK
     assert call(N=0, X=None, W=None, s=None, z=None, Y=None) == OK
+
+
+def test_mxfp4_validates_before_launch(L):
+    BF16, U8 = 1, 3
+    assert L.hqq_mxfp4_quantize(FAKE, BF16, 4, 48, FAKE, FAKE, None) == SHAPE
+    assert L.hqq_mxfp4_quantize(FAKE, U8, 4, 64, FAKE, FAKE, None) == UNSUPPORTED
+    assert L.hqq_mxfp4_quantize(FAKE, BF16, -1, 64, FAKE, FAKE, None) == INVALID
+    assert L.hqq_mxfp4_quantize(None, BF16, 4, 64, FAKE, FAKE, None) == INVALID
+    assert L.hqq_mxfp4_quantize(FAKE_ODD, BF16, 4, 64, FAKE, FAKE, None) == ALIGN
+    assert L.hqq_mxfp4_quantize(None, BF16, 0, 64, None, None, None) == OK
+    assert L.hqq_mxfp4_dequantize(FAKE, FAKE, 4, 40, BF16, FAKE, None) == SHAPE
+    assert L.hqq_mxfp4_dequantize(FAKE, FAKE, 4, 64, BF16, FAKE + 8, None) == ALIGN
+    assert L.hqq_mxfp4_dequantize(FAKE, FAKE, 4, 64, U8, FAKE, None) == UNSUPPORTED
+    assert L.hqq_mxfp4_dequantize(None, None, 4, 0, BF16, None, None) == OK
