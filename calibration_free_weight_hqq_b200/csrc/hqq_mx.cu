@@ -26,7 +26,11 @@
 namespace hqqk {
 namespace {
 
+#ifndef HQQ_MX_UNROLL
+#define HQQ_MX_UNROLL 4
+#endif
 constexpr int kMxThreads = 256;
+constexpr int kMxUnroll = HQQ_MX_UNROLL;  // 256-element chunks per warp per iteration
 
 template <int DT>
 __device__ __forceinline__ void load8(const void* W, int64_t i, float (&v)[8]) {
@@ -90,6 +94,29 @@ __device__ __forceinline__ __half2 e2m1x2_to_half2(uint32_t byte) {
   return *reinterpret_cast<__half2*>(&h);
 }
 
+// Encode the 8 elements v of one lane (its block = 4 lanes) and store them.
+__device__ __forceinline__ void encode8(const float (&v)[8], int64_t i, bool in,
+                                        uint8_t* __restrict__ codes,
+                                        uint8_t* __restrict__ scales, int lane) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(v[k]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+  const int e = mx_exponent(amax);
+  const float inv = pow2i(-e);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    packed |= e2m1x2(__fmul_rn(v[2 * k], inv), __fmul_rn(v[2 * k + 1], inv)) << (8 * k);
+  if (in) {
+    *reinterpret_cast<uint32_t*>(codes + i / 2) = packed;
+    if ((lane & 3) == 0) scales[i / 32] = static_cast<uint8_t>(e + 127);
+  }
+}
+
+// Each warp takes kMxUnroll consecutive 256-element chunks per iteration and issues all their
+// loads before converting any (more bytes in flight per SM).
 template <int DT>
 __global__ void __launch_bounds__(kMxThreads) mxfp4_quantize_kernel(const void* __restrict__ W,
                                                                      int64_t n,
@@ -98,30 +125,22 @@ __global__ void __launch_bounds__(kMxThreads) mxfp4_quantize_kernel(const void* 
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-       w * 256 < n; w += nwarps) {
-    const int64_t i = w * 256 + lane * 8;
-    const bool in = i < n;  // n % 32 == 0: the 4 lanes of a block are all in or all out
-    float v[8];
-    if (in) {
-      load8<DT>(W, i, v);
-    } else {
+       w * 256 * kMxUnroll < n; w += nwarps) {
+    float v[kMxUnroll][8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = 0.0f;
+    for (int u = 0; u < kMxUnroll; ++u) {
+      const int64_t i = (w * kMxUnroll + u) * 256 + lane * 8;
+      if (i < n) {  // n % 32 == 0: the 4 lanes of a block are all in or all out
+        load8<DT>(W, i, v[u]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[u][k] = 0.0f;
+      }
     }
-    float amax = 0.0f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(v[k]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-    const int e = mx_exponent(amax);
-    const float inv = pow2i(-e);
-    uint32_t packed = 0;
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      packed |= e2m1x2(__fmul_rn(v[2 * k], inv), __fmul_rn(v[2 * k + 1], inv)) << (8 * k);
-    if (in) {
-      *reinterpret_cast<uint32_t*>(codes + i / 2) = packed;
-      if ((lane & 3) == 0) scales[i / 32] = static_cast<uint8_t>(e + 127);
+    for (int u = 0; u < kMxUnroll; ++u) {
+      const int64_t i = (w * kMxUnroll + u) * 256 + lane * 8;
+      encode8(v[u], i, i < n, codes, scales, lane);
     }
   }
 }
@@ -133,32 +152,42 @@ __global__ void __launch_bounds__(kMxThreads) mxfp4_dequantize_kernel(
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-       w * 256 < n; w += nwarps) {
-    const int64_t i = w * 256 + lane * 8;
-    if (i >= n) continue;
-    const uint32_t c = __ldcs(reinterpret_cast<const unsigned int*>(codes + i / 2));
-    const float x = pow2i(static_cast<int>(__ldg(scales + i / 32)) - 127);
-    float v[8];
+       w * 256 * kMxUnroll < n; w += nwarps) {
+    uint32_t c[kMxUnroll];
+    int sc[kMxUnroll];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = __half22float2(e2m1x2_to_half2((c >> (8 * k)) & 0xFFu));
-      v[2 * k] = __fmul_rn(f.x, x);  // exact: an E2M1 value times a power of two
-      v[2 * k + 1] = __fmul_rn(f.y, x);
+    for (int u = 0; u < kMxUnroll; ++u) {
+      const int64_t i = (w * kMxUnroll + u) * 256 + lane * 8;
+      c[u] = i < n ? __ldcs(reinterpret_cast<const unsigned int*>(codes + i / 2)) : 0u;
+      sc[u] = i < n ? static_cast<int>(__ldg(scales + i / 32)) : 127;
     }
-    if constexpr (OUT == kF32) {
-      float4* p = reinterpret_cast<float4*>(static_cast<float*>(out) + i);
-      __stcs(p, make_float4(v[0], v[1], v[2], v[3]));
-      __stcs(p + 1, make_float4(v[4], v[5], v[6], v[7]));
-    } else {
-      const uint4 o = make_uint4(pack2_16<OUT>(v[0], v[1]), pack2_16<OUT>(v[2], v[3]),
-                                 pack2_16<OUT>(v[4], v[5]), pack2_16<OUT>(v[6], v[7]));
-      __stcs(reinterpret_cast<uint4*>(static_cast<unsigned short*>(out) + i), o);
+#pragma unroll
+    for (int u = 0; u < kMxUnroll; ++u) {
+      const int64_t i = (w * kMxUnroll + u) * 256 + lane * 8;
+      if (i >= n) continue;
+      const float x = pow2i(sc[u] - 127);
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(e2m1x2_to_half2((c[u] >> (8 * k)) & 0xFFu));
+        v[2 * k] = __fmul_rn(f.x, x);  // exact: an E2M1 value times a power of two
+        v[2 * k + 1] = __fmul_rn(f.y, x);
+      }
+      if constexpr (OUT == kF32) {
+        float4* p = reinterpret_cast<float4*>(static_cast<float*>(out) + i);
+        __stcs(p, make_float4(v[0], v[1], v[2], v[3]));
+        __stcs(p + 1, make_float4(v[4], v[5], v[6], v[7]));
+      } else {
+        const uint4 o = make_uint4(pack2_16<OUT>(v[0], v[1]), pack2_16<OUT>(v[2], v[3]),
+                                   pack2_16<OUT>(v[4], v[5]), pack2_16<OUT>(v[6], v[7]));
+        __stcs(reinterpret_cast<uint4*>(static_cast<unsigned short*>(out) + i), o);
+      }
     }
   }
 }
 
 unsigned mx_grid(int64_t n) {
-  const int64_t warps = (n + 255) / 256;
+  const int64_t warps = (n + 256 * kMxUnroll - 1) / (256 * kMxUnroll);
   const int64_t blocks = (warps + kMxThreads / 32 - 1) / (kMxThreads / 32);
   return static_cast<unsigned>(blocks < 148 * 16 ? blocks : 148 * 16);
 }
