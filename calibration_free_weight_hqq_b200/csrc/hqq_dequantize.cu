@@ -263,6 +263,46 @@ __global__ void __launch_bounds__(kDBlock, HQQ_DQ_MINB)
   }
 }
 
+// 4-bit codes, plain (not second-level) meta, 16-bit output - the layout every bench step
+// and the linear layer use. A warp covers 256 consecutive elements per chunk (lane l: elements
+// 8l .. 8l+7, one 32-bit code load, one 16-byte store), kD4Unroll chunks per warp per tile;
+// all of a tile's loads are issued before any conversion, which keeps more bytes in flight
+// than the generic kernel's two 8-element chunks per thread.
+constexpr int kD4Unroll = 4;
+constexpr int64_t kDTile4 = (int64_t)kDBlock * 8 * kD4Unroll;
+
+template <int OUT_DT, int MAXB>
+__global__ void __launch_bounds__(kDBlock) dequant4_axis1_kernel(
+    const __grid_constant__ DBatch<MAXB> batch) {
+  const int64_t total = batch.tile_start[batch.n];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+    int64_t local;
+    const DArgs a = batch_args(batch, t, &local);
+    const int64_t base = local * kDTile4 + (int64_t)warp * (kD4Unroll * 256) + lane * 8;
+    uint32_t w[kD4Unroll];
+    float sc[kD4Unroll], zr[kD4Unroll];
+#pragma unroll
+    for (int u = 0; u < kD4Unroll; ++u) {
+      const int64_t i = base + u * 256;
+      if (i < a.n) {  // n and G are multiples of 8: a lane's 8 elements share one group
+        w[u] = __ldcs(reinterpret_cast<const unsigned int*>(a.packed + i / 2));
+        const int64_t g = i >> a.log2_group;
+        sc[u] = load_meta(a.scale, a.meta_dtype, g);
+        zr[u] = load_meta(a.zero, a.meta_dtype, g);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kD4Unroll; ++u) {
+      const int64_t i = base + u * 256;
+      if (i < a.n)
+        st_out(reinterpret_cast<uint4*>(reinterpret_cast<unsigned short*>(a.out) + i),
+               dequant8_4bit<OUT_DT>(w[u], make_float2(-zr[u], -zr[u]),
+                                     make_float2(sc[u], sc[u])));
+    }
+  }
+}
+
 // axis=0 (groups run down columns): element (r, c) is code j = r % G of group
 // g = (r / G)*cols + c. Rows with cols % 8 == 0 take 8 columns per thread; a block covers
 // one tile of kDBlock*8 elements of one matrix.
@@ -355,6 +395,21 @@ static void fill_dbatch(const DequantJob* jobs, int n, int64_t tile_elems, DBatc
 template <int NB, int OUT_DT, int MAXB>
 static cudaError_t launch_nb_dt(const DequantJob* jobs, int n, cudaStream_t st) {
   DBatch<MAXB> b;
+  if constexpr (NB == 4 && OUT_DT != kF32) {
+    bool plain_meta = jobs[0].axis == 1;
+    for (int i = 0; i < n; ++i) plain_meta = plain_meta && !jobs[i].scale_mm && !jobs[i].zero_mm;
+    if (plain_meta) {
+      fill_dbatch<MAXB>(jobs, n, kDTile4, &b);
+      const int64_t tiles = b.tile_start[b.n];
+      if (tiles == 0) return cudaSuccess;
+      int resident = 0;
+      const cudaError_t e = resident_blocks(dequant4_axis1_kernel<OUT_DT, MAXB>, &resident);
+      if (e != cudaSuccess) return e;
+      const int64_t blocks = tiles < resident ? tiles : resident;
+      dequant4_axis1_kernel<OUT_DT, MAXB><<<(unsigned)blocks, kDBlock, 0, st>>>(b);
+      return cudaGetLastError();
+    }
+  }
   if (jobs[0].axis == 1) {
     fill_dbatch<MAXB>(jobs, n, kDTile1, &b);
     const int64_t tiles = b.tile_start[b.n];

@@ -96,4 +96,26 @@ __device__ __forceinline__ uint32_t pack2_16(float a, float b) {
   }
 }
 
+// Eight consecutive 4-bit codes (LSB-first in a little-endian word: code 2b in the low
+// nibble of byte b, code 2b+1 in its high nibble) to eight dequantized 16-bit values of type
+// OUT (kBF16 or kF16): (float(q) - zero) * scale with the dequantizer's three roundings. Each
+// code becomes the float 2^23 + q by placing its byte under the exponent bits (0x4B000000);
+// subtracting 2^23 is exact; q - zero is computed as q + (-zero) (identical rounding). The
+// arithmetic runs on fp32 pairs (sm_100 FADD2/FMUL2: one instruction, two lanes, the same
+// rounding as two scalar operations).
+template <int OUT>
+__device__ __forceinline__ uint4 dequant8_4bit(uint32_t w, float2 neg_zero, float2 scale) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+  const float2 neg_magic = make_float2(-8388608.0f, -8388608.0f);
+  uint32_t o[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const float2 m = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7540 + b)),
+                                 __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7540 + b)));
+    const float2 v = __fmul2_rn(__fadd2_rn(__fadd2_rn(m, neg_magic), neg_zero), scale);
+    o[b] = pack2_16<OUT>(v.x, v.y);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 }  // namespace hqqk

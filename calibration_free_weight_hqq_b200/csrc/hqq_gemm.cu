@@ -220,29 +220,13 @@ __device__ __forceinline__ uint32_t mma_idesc() {
          (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
-// Eight consecutive 4-bit codes (LSB-first in a little-endian word: code 2b in the low
-// nibble of byte b, code 2b+1 in its high nibble) to eight dequantized 16-bit values.
-// Each code becomes the float 2^23 + q by placing its byte under the exponent bits
-// (0x4B000000); subtracting 2^23 is exact. Then (q - zero)·scale with two roundings and one
-// final rounding to the 16-bit type, as the dequantizer computes it.
-// The arithmetic runs on fp32 pairs (sm_100 packed FADD2/FMUL2: one instruction for two
-// lanes of the same rounding), q - zero as q + (-zero), which rounds identically.
+// The 4-bit conversion of the operand tile is dequant8_4bit (hqq_device.cuh): the same three
+// roundings as hqq_dequantize.
 template <bool F16>
 __device__ __forceinline__ uint4 dequant8(uint32_t w, float2 neg_zero, float2 scale) {
-  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-  const float2 neg_magic = make_float2(-8388608.0f, -8388608.0f);
-  uint32_t o[4];
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    const float2 m = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7540 + b)),
-                                 __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7540 + b)));
-    const float2 v = __fmul2_rn(__fadd2_rn(__fadd2_rn(m, neg_magic), neg_zero), scale);
-    o[b] = pack2_16<F16 ? kF16 : kBF16>(v.x, v.y);
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
+  return dequant8_4bit<F16 ? kF16 : kBF16>(w, neg_zero, scale);
 }
 
-// Meta values of type MT as raw bits and as fp32.
 template <int MT>
 __device__ __forceinline__ uint32_t meta_load(const uint8_t* p) {
   if constexpr (MT == kF32) return __ldg(reinterpret_cast<const unsigned int*>(p));
