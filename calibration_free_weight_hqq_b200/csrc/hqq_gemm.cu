@@ -8,20 +8,13 @@
 // the activation dtype exactly as hqq_dequantize writes it; Y[m, n] = dtype(Σ_k X[m,k]·W'[n,k]
 // accumulated in fp32 (+ bias[n])).
 //
-// Blackwell design, one 256 x 256 output tile per CTA, 64 + 32*HQQ_GEMM_DQ_WARPS threads, one
-// CTA per SM:
-//   warp 0      TMA producer: X tile (two 128 x 64 boxes, 128-byte swizzle, which is the UMMA
-//               K-major SW128 layout) and the packed-code tile (256 rows x 32 bytes) into a
-//               3-stage ring.
-//   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators); lane 0 issues
-//               tcgen05.mma (kind::f16, M=128, N=256, K=16) - 8 per k-block - and releases
-//               ring slots with tcgen05.commit.
-//   warps 2-    dequantize: (scale, zero) of their rows fetched 8 k-blocks ahead (one group
-//               per row per k-block: BK = 64 = group size), 4-bit codes to bf16/fp16 straight
-//               into a 2-stage ring in the SW128 K-major layout
-//               (16-byte stores, conflict-free); after the last k-block, the epilogue:
-//               tcgen05.ld of the accumulators, bias, rounding, 32 x 32 blocks staged in
-//               shared memory and written by TMA stores.
+// Two kernels, picked by the number of rows M of X (tokens):
+//   * w4a16_gemm_2sm_kernel (M > 128): a CTA pair computes a 512 x 256 output tile with the
+//     2-SM tensor-core MMA; each CTA dequantizes its own 128 rows of the W' tile (description
+//     at the kernel).
+//   * w4a16_skinny_kernel (M <= 128, decode-sized batches): the roles swap - W' (128 rows per
+//     CTA) is the MMA's M operand and the tokens its N - and a cluster of 8 CTAs splits K,
+//     reducing the partial sums over distributed shared memory (description at the kernel).
 // Every wait is bounded (about two seconds of %globaltimer); on expiry the CTA raises an abort
 // flag, counts a timeout in g_gemm_timeouts, skips its remaining work, waits (bounded) for
 // its own asynchronous operations and frees its TMEM.
@@ -32,6 +25,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <mutex>
 #include <type_traits>
 
@@ -44,48 +38,12 @@ __device__ unsigned int g_gemm_timeouts = 0;
 
 namespace {
 
-#ifndef HQQ_GEMM_DQ_WARPS
-#define HQQ_GEMM_DQ_WARPS 16
-#endif
-#ifndef HQQ_GEMM_B_STAGES
-#define HQQ_GEMM_B_STAGES 2
-#endif
-#ifndef HQQ_GEMM_TMA_STORE
-#define HQQ_GEMM_TMA_STORE 1
-#endif
-#ifndef HQQ_GEMM_2SM
-#define HQQ_GEMM_2SM 1
-#endif
-
-constexpr int kBM = 256, kBN = 256, kBK = 64;
-constexpr int kStagesL = 3;                  // X + packed codes + meta
-constexpr int kStagesB = HQQ_GEMM_B_STAGES;  // dequantized operand
-constexpr int kDqWarps = HQQ_GEMM_DQ_WARPS;  // 8 or 16
-static_assert(kDqWarps == 8 || kDqWarps == 16, "dequantize warps");
-constexpr int kDqIters = kBN * (kBK / 8) / (32 * kDqWarps);  // 8-code chunks per thread
-constexpr int kThreads = 64 + 32 * kDqWarps;
-constexpr uint32_t kAHalf = 128 * kBK * 2;
-constexpr uint32_t kABytes = 2 * kAHalf;
-constexpr uint32_t kPBytes = kBN * kBK / 2;
-constexpr uint32_t kBBytes = kBN * kBK * 2;
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffB = kOffA + kStagesL * kABytes;
-constexpr uint32_t kOffP = kOffB + kStagesB * kBBytes;
-constexpr uint32_t kOffBar = kOffP + kStagesL * kPBytes;
+constexpr int kBN = 256, kBK = 64;  // W' rows per 2-SM pair tile; K per k-block = group size
 // Epilogue staging (reuses the X ring once the last MMA has completed): per dequantize warp two
 // 32 x 32 output blocks of 64-byte rows, stored by TMA.
 constexpr uint32_t kStageBytes = 32 * 32 * 2;
-static_assert(kDqWarps * 2 * kStageBytes <= kStagesL * kABytes, "staging fits the X ring");
-constexpr int kBarFullL = 0, kBarEmptyL = kStagesL, kBarFullB = 2 * kStagesL,
-              kBarEmptyB = 2 * kStagesL + kStagesB, kBarAcc = 2 * kStagesL + 2 * kStagesB;
-constexpr int kNumBars = kBarAcc + 1;
-constexpr uint32_t kOffTmem = kOffBar + 8 * kNumBars;
-constexpr uint32_t kOffAbort = kOffTmem + 4;
-constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;  // + slack to align the base to 1024
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
-static_assert(kOffB % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0, "SW128 tiles");
-static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 struct GemmArgs {
   const void* scale;
@@ -236,275 +194,6 @@ template <int MT>
 __device__ __forceinline__ float meta_f32(uint32_t h) {
   if constexpr (MT == kF32) return __uint_as_float(h);
   return MT == kBF16 ? bf16_bits_to_f32(h) : f16_bits_to_f32(h);
-}
-
-template <bool F16, int MT>
-__global__ void __launch_bounds__(kThreads, 1)
-    w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                      const __grid_constant__ CUtensorMap tmap_w,
-                      const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const uint32_t sbase = smem_u32(smem);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
-  const int KB = args.K / kBK;
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + kOffAbort);
-  auto bar = [&](int i) { return sbase + kOffBar + 8u * static_cast<uint32_t>(i); };
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStagesL; ++s) {
-      mbar_init(bar(kBarFullL + s), 1);  // producer's expect_tx (+ the copies' bytes)
-      mbar_init(bar(kBarEmptyL + s), 1);  // MMA commit
-    }
-    for (int t = 0; t < kStagesB; ++t) {
-      mbar_init(bar(kBarFullB + t), kDqWarps);
-      mbar_init(bar(kBarEmptyB + t), 1);
-    }
-    mbar_init(bar(kBarAcc), 1);
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_y)) : "memory");
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     sbase + kOffTmem),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer (TMA only)
-    int issued = 0;
-    for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % kStagesL;
-      const uint32_t ph = (kb / kStagesL) & 1;
-      if (!mbar_wait(bar(kBarEmptyL + s), ph ^ 1, abort_flag)) break;
-      if (lane == 0) {
-        const uint32_t full = bar(kBarFullL + s);
-        mbar_arrive_tx(full, kABytes + kPBytes);
-        const uint32_t a = sbase + kOffA + s * kABytes;
-        tma_load_2d(a, &tmap_x, kb * kBK, m0, full);
-        tma_load_2d(a + kAHalf, &tmap_x, kb * kBK, m0 + 128, full);
-        tma_load_2d(sbase + kOffP + s * kPBytes, &tmap_w, kb * (kBK / 2), n0, full);
-      }
-      ++issued;
-    }
-    // Before leaving, make sure no copy of ours is still landing in shared memory: wait for
-    // the last use of every slot (already complete on the normal path).
-    if (lane == 0) {
-      for (int kb = issued - 1; kb >= 0 && kb >= issued - kStagesL; --kb) {
-        const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(bar(kBarFullL + kb % kStagesL), (kb / kStagesL) & 1) &&
-               globaltimer() - t0 < kWaitLimitNs) {
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = mma_idesc<F16>();
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % kStagesL, t = kb % kStagesB;
-        if (!mbar_wait(bar(kBarFullL + s), (kb / kStagesL) & 1, abort_flag)) break;
-        if (!mbar_wait(bar(kBarFullB + t), (kb / kStagesB) & 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t a = sbase + kOffA + s * kABytes;
-        const uint64_t da0 = sw128_kmajor_desc(a), da1 = sw128_kmajor_desc(a + kAHalf);
-        const uint64_t db = sw128_kmajor_desc(sbase + kOffB + t * kBBytes);
-#pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          // K step of 16 elements = 32 bytes inside the swizzled 128-byte row.
-          const uint32_t acc = (kb | k) != 0;
-          tc_mma(tmem, da0 + 2 * k, db + 2 * k, idesc, acc);
-          tc_mma(tmem + kBN, da1 + 2 * k, db + 2 * k, idesc, acc);
-        }
-        tc_commit(bar(kBarEmptyL + s));
-        tc_commit(bar(kBarEmptyB + t));
-      }
-      tc_commit(bar(kBarAcc));  // also the last word on any aborted run
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ dequantize
-    // Thread (d, lane) converts 8-code chunk `chunk` of rows d*4*kDqIters + 4j + lane/8. The
-    // 8 lanes that share a row also share its (scale, zero): each fetches the values of one
-    // of the next 8 k-blocks (lane & 7 = offset) from global memory a full 8 k-blocks ahead,
-    // and every k-block the value is taken from the lane that holds it with a shuffle. For
-    // 16-bit meta scale and zero travel packed in one word.
-    const int d = warp - 2;
-    const int chunk = lane & 7;
-    constexpr int kMB = MT == kF32 ? 4 : 2;
-    constexpr int kWords = MT == kF32 ? 2 : 1;  // shuffled words per row and k-block
-    const int64_t groups_per_row = args.K / kBK;
-    const uint8_t* row_s[kDqIters];
-    const uint8_t* row_z[kDqIters];
-#pragma unroll
-    for (int j = 0; j < kDqIters; ++j) {
-      const int n = n0 + d * (4 * kDqIters) + j * 4 + (lane >> 3);
-      const int64_t off = static_cast<int64_t>(n) * groups_per_row * kMB;
-      row_s[j] = n < args.N ? static_cast<const uint8_t*>(args.scale) + off : nullptr;
-      row_z[j] = n < args.N ? static_cast<const uint8_t*>(args.zero) + off : nullptr;
-    }
-    uint32_t nxt_s[kDqIters], nxt_z[kDqIters], cur[kDqIters][kWords];
-    auto fetch8 = [&](int kb8) {  // this lane's k-block of the 8-block window kb8
-      const int kk = kb8 * 8 + chunk;
-#pragma unroll
-      for (int j = 0; j < kDqIters; ++j) {
-        const bool in = row_s[j] != nullptr && kk < KB;  // rows past N dequantize to 0
-        nxt_s[j] = in ? meta_load<MT>(row_s[j] + static_cast<int64_t>(kk) * kMB) : 0u;
-        nxt_z[j] = in ? meta_load<MT>(row_z[j] + static_cast<int64_t>(kk) * kMB) : 0u;
-      }
-    };
-    if (KB > 0) fetch8(0);
-    for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % kStagesL, t = kb % kStagesB;
-      if ((kb & 7) == 0) {  // the window's values arrived during the previous 8 k-blocks
-#pragma unroll
-        for (int j = 0; j < kDqIters; ++j) {
-          if constexpr (kWords == 1) {
-            cur[j][0] = nxt_s[j] | (nxt_z[j] << 16);
-          } else {
-            cur[j][0] = nxt_s[j];
-            cur[j][kWords - 1] = nxt_z[j];
-          }
-        }
-        if (kb + 8 < KB) fetch8((kb >> 3) + 1);
-      }
-      const int src = (lane & ~7) | (kb & 7);
-      float sc[kDqIters], nz[kDqIters];
-#pragma unroll
-      for (int j = 0; j < kDqIters; ++j) {
-        if constexpr (kWords == 1) {
-          const uint32_t v = __shfl_sync(0xFFFFFFFFu, cur[j][0], src);
-          sc[j] = meta_f32<MT>(v & 0xFFFFu);
-          nz[j] = -meta_f32<MT>(v >> 16);
-        } else {
-          sc[j] = meta_f32<MT>(__shfl_sync(0xFFFFFFFFu, cur[j][0], src));
-          nz[j] = -meta_f32<MT>(__shfl_sync(0xFFFFFFFFu, cur[j][kWords - 1], src));
-        }
-      }
-      // warp-uniform outcome: the shuffles above and below take every lane
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(kBarFullL + s), (kb / kStagesL) & 1, abort_flag)))
-        break;
-      if (!__all_sync(0xFFFFFFFFu,
-                      mbar_wait(bar(kBarEmptyB + t), ((kb / kStagesB) & 1) ^ 1, abort_flag)))
-        break;
-      const uint8_t* P = smem + kOffP + s * kPBytes;
-      uint8_t* B = smem + kOffB + t * kBBytes;
-      uint32_t w[kDqIters];
-#pragma unroll
-      for (int j = 0; j < kDqIters; ++j) {
-        const int row = d * (4 * kDqIters) + j * 4 + (lane >> 3);
-        w[j] = *reinterpret_cast<const uint32_t*>(P + row * 32 + chunk * 4);
-      }
-#pragma unroll
-      for (int j = 0; j < kDqIters; ++j) {
-        const int row = d * (4 * kDqIters) + j * 4 + (lane >> 3);
-        *reinterpret_cast<uint4*>(B + row * 128 + ((chunk ^ (row & 7)) << 4)) =
-            dequant8<F16>(w[j], make_float2(nz[j], nz[j]), make_float2(sc[j], sc[j]));
-      }
-      fence_proxy_async_smem();  // generic-proxy writes -> read by the tensor core
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarFullB + t));
-    }
-
-    // ------------------------------------------------------------ epilogue
-    // 4 consecutive warps cover the four TMEM lane quarters; groups of four alternate
-    // between the two accumulators and split the 8 column chunks between them
-    constexpr int kChunksPerWarp = (kBN / 32) * 8 / kDqWarps;
-    const int h = (d >> 2) & 1;    // which 128-row accumulator
-    const int c0 = (d >> 3) * kChunksPerWarp;
-    const int quarter = warp & 3;  // TMEM lanes this warp may read: 32*quarter ..
-    // warp-uniform: tcgen05.ld below is a .sync.aligned instruction
-    const bool ok =
-        __all_sync(0xFFFFFFFFu, mbar_wait(bar(kBarAcc), 0, abort_flag) && !*abort_flag);
-    tc_fence_after();
-    const int row0 = m0 + h * 128 + quarter * 32;
-    const unsigned short* bias = reinterpret_cast<const unsigned short*>(args.bias);
-#if HQQ_GEMM_TMA_STORE
-    uint8_t* stage0 = smem + kOffA + static_cast<uint32_t>(d) * 2u * kStageBytes;
-#else
-    const int m = row0 + lane;
-    typedef typename std::conditional<F16, __half, __nv_bfloat16>::type T;
-    T* Yrow = reinterpret_cast<T*>(args.Y) + static_cast<int64_t>(m) * args.N;
-#endif
-#pragma unroll 1
-    for (int c = c0; c < c0 + kChunksPerWarp; ++c) {
-      uint32_t r[32];
-      if (ok && KB > 0) {
-        tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + h * kBN + c * 32, r);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = 0u;  // empty sum (K = 0)
-      }
-      const int nc = n0 + c * 32;
-      uint32_t o[16];
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float v0 = __uint_as_float(r[i]), v1 = __uint_as_float(r[i + 1]);
-        if (bias != nullptr && nc + i < args.N) {  // N % 8 == 0: pairs never straddle
-          v0 = __fadd_rn(v0, F16 ? f16_bits_to_f32(bias[nc + i]) : bf16_bits_to_f32(bias[nc + i]));
-          v1 = __fadd_rn(v1, F16 ? f16_bits_to_f32(bias[nc + i + 1])
-                                 : bf16_bits_to_f32(bias[nc + i + 1]));
-        }
-        o[i / 2] = pack2_16<F16 ? kF16 : kBF16>(v0, v1);
-      }
-#if HQQ_GEMM_TMA_STORE
-      // Stage the warp's 32 x 32 block (row = lane, 64 bytes) in the 64-byte swizzle the
-      // output tensor map uses (16-byte chunk q of row r at chunk q ^ ((r >> 1) & 3)), which
-      // makes the four 16-byte stores conflict-free; one lane then stores it with TMA.
-      // Rows past M and columns past N are clipped by the copy itself.
-      uint8_t* stage = stage0 + ((c - c0) & 1) * kStageBytes;
-      if (lane == 0 && c - c0 >= 2) bulk_wait_read<1>();  // this buffer's previous store
-      __syncwarp();
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(stage + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) =
-            make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0 && ok) {
-        tma_store_2d(&tmap_y, smem_u32(stage), nc, row0);
-        bulk_commit();
-      }
-#else
-      if (!ok || m >= args.M || nc >= args.N) continue;
-      if (nc + 32 <= args.N) {
-        uint4* dst = reinterpret_cast<uint4*>(Yrow + nc);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (nc + 2 * i < args.N) reinterpret_cast<uint32_t*>(Yrow + nc)[i] = o[i];
-      }
-#endif
-    }
-#if HQQ_GEMM_TMA_STORE
-    if (lane == 0) bulk_wait_read<0>();  // shared memory stays ours until the stores read it
-    __syncwarp();
-#endif
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kTmemCols)
-                 : "memory");
-  }
 }
 
 // ================================================================ 2-SM kernel
@@ -911,6 +600,332 @@ __global__ void __launch_bounds__(sm2::kThreads, 1)
   }
 }
 
+// ================================================================ skinny kernel (M <= 128)
+// Decode-sized batches: too few output tiles for the 2-SM kernel to fill the GPU, and the
+// weight is read once per token batch, so the work is the dequantization of W' and its HBM
+// read. Roles swap: D[n, m] = sum_k W'[n, k] * X[m, k] with W' (128 rows per CTA, dequantized
+// into shared memory in the SW128 K-major layout) as the MMA's A operand (M = 128) and the
+// ntok <= 128 token rows of X (TMA, SW128) as its B operand (N = ntok, a multiple of 16); the
+// accumulator is 128 TMEM lanes x ntok columns. A cluster of kSkS CTAs shares one W' row tile
+// and splits K into contiguous slices; after its slice each CTA reads its partial D and writes
+// rows 16r .. 16r+15 of it into a per-source slot of cluster CTA r (distributed shared memory,
+// plain stores); after a cluster barrier CTA r sums its kSkS slots in rank order (fixed order:
+// deterministic), adds bias, rounds and stores its 16 output rows for every token.
+namespace skinny {
+constexpr int kS = 4;            // CTAs per cluster = K slices
+constexpr int kRows = 128;       // W' rows per CTA
+constexpr int kTokMax = 64;      // tokens per CTA (MMA N); larger batches take several tiles
+constexpr int kMaxM = 128;       // the skinny kernel serves M <= kMaxM
+constexpr int kSub = 4;          // k-blocks per load stage: 128-byte rows of packed codes
+constexpr int kStagesL = 2;      // load stages (X boxes + packed codes of kSub k-blocks)
+constexpr int kStagesB = 3;      // dequantized W' stages, one k-block each
+constexpr int kDqWarps = 8;
+constexpr int kDqIters = kRows * (kBK / 8) / (32 * kDqWarps);  // chunks per thread
+constexpr int kThreads = 64 + 32 * kDqWarps;
+constexpr uint32_t kPBytes = kRows * kBK / 2 * kSub;  // 16 KB: 128 rows x 128 bytes
+constexpr uint32_t kWBytes = kRows * kBK * 2;      // 16 KB
+constexpr int kOwnRows = kRows / kS;                // output rows reduced per CTA
+constexpr int kFullL = 0, kEmptyL = kStagesL, kFullW = 2 * kStagesL, kEmptyW = kFullW + kStagesB,
+              kAcc = kEmptyW + kStagesB;
+constexpr int kNumBars = kAcc + 1;
+constexpr uint32_t kTmemCols = 128;
+// Shared-memory layout for ntok tokens (a multiple of 16): the X ring holds ntok rows per stage
+// and the reduction slots ntok columns, so small batches leave room for two CTAs per SM.
+struct Layout {
+  uint32_t x_stage, off_w, off_p, off_red, slot, off_bar, off_tmem, off_abort, bytes;
+};
+__host__ __device__ constexpr Layout layout(int ntok) {
+  Layout L{};
+  L.x_stage = static_cast<uint32_t>(ntok) * kBK * 2 * kSub;  // kSub SW128 boxes of ntok rows
+  L.off_w = kStagesL * L.x_stage;
+  L.off_p = L.off_w + kStagesB * kWBytes;
+  L.off_red = L.off_p + kStagesL * kPBytes;
+  L.slot = static_cast<uint32_t>(kOwnRows) * static_cast<uint32_t>(ntok) * 4;
+  L.off_bar = L.off_red + kS * L.slot;
+  L.off_tmem = L.off_bar + 8 * kNumBars;
+  L.off_abort = L.off_tmem + 4;
+  L.bytes = L.off_abort + 4 + 1024;  // + slack to align the base to 1024
+  return L;
+}
+static_assert(kWBytes % 1024 == 0, "SW128 tiles");
+static_assert(layout(kTokMax).bytes <= 232448, "shared memory per CTA");
+}  // namespace skinny
+
+// Instruction descriptor of kind::f16, M = 128, N = ntok (a multiple of 16, <= 256).
+template <bool F16>
+__device__ __forceinline__ uint32_t mma_idesc_m128(int ntok) {
+  constexpr uint32_t fmt = F16 ? 0u : 1u;
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | (static_cast<uint32_t>(ntok >> 3) << 17) |
+         (static_cast<uint32_t>(128 >> 4) << 24);
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11,"
+      " %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void st_cluster_v4f(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+template <bool F16, int MT>
+__global__ void __launch_bounds__(skinny::kThreads, 2)
+    w4a16_skinny_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                        const __grid_constant__ CUtensorMap tmap_w, const GemmArgs args,
+                        int ntok) {
+  // this kernel's layout (shadows the 2-SM kernel's constants)
+  constexpr int kS = skinny::kS, kStagesL = skinny::kStagesL, kStagesB = skinny::kStagesB;
+  constexpr int kSub = skinny::kSub;
+  constexpr int kDqWarps = skinny::kDqWarps, kDqIters = skinny::kDqIters;
+  constexpr int kOwnRows = skinny::kOwnRows, kTokMax = skinny::kTokMax;
+  constexpr uint32_t kPBytes = skinny::kPBytes, kWBytes = skinny::kWBytes;
+  const skinny::Layout lay = skinny::layout(ntok);
+  const uint32_t kXBytes = lay.x_stage, kSlotBytes = lay.slot;
+  const uint32_t kOffX = 0, kOffW = lay.off_w, kOffP = lay.off_p, kOffRed = lay.off_red,
+                 kOffBar = lay.off_bar, kOffTmem = lay.off_tmem, kOffAbort = lay.off_abort;
+  constexpr int kFullL = skinny::kFullL, kEmptyL = skinny::kEmptyL, kFullW = skinny::kFullW,
+                kEmptyW = skinny::kEmptyW, kAcc = skinny::kAcc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();  // K slice of this CTA; also which 16 rows it reduces
+  const int n0 = static_cast<int>(blockIdx.x / kS) * skinny::kRows;
+  const int m0 = blockIdx.y * kTokMax;
+  const int KB = args.K / kBK;
+  const int per = (KB + kS - 1) / kS;
+  const int kb0 = min(KB, static_cast<int>(rank) * per), kb1 = min(KB, kb0 + per);
+  const int nkb = kb1 - kb0;
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + kOffAbort);
+  auto bar = [&](int i) { return sbase + kOffBar + 8u * static_cast<uint32_t>(i); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStagesL; ++s) {
+      mbar_init(bar(kFullL + s), 1);
+      mbar_init(bar(kEmptyL + s), 1);
+    }
+    for (int t = 0; t < kStagesB; ++t) {
+      mbar_init(bar(kFullW + t), kDqWarps);
+      mbar_init(bar(kEmptyW + t), 1);
+    }
+    mbar_init(bar(kAcc), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     sbase + kOffTmem),
+                 "r"(skinny::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // every CTA of the cluster is running before anyone writes into another
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
+  const uint32_t xbox = static_cast<uint32_t>(ntok) * kBK * 2;  // one X box (one k-block)
+  const int nsb = (nkb + kSub - 1) / kSub;                        // load stages of the slice
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    // one stage = kSub k-blocks: kSub X boxes and one box of 128 packed-code rows x 128 bytes
+    // (boxes reaching past K read zeros; k-blocks past the slice are loaded but not used)
+    int issued = 0;
+    for (int j = 0; j < nsb; ++j) {
+      const int s = j % kStagesL, kb = kb0 + j * kSub;
+      if (!mbar_wait(bar(kEmptyL + s), ((j / kStagesL) & 1) ^ 1, abort_flag)) break;
+      if (lane == 0) {
+        const uint32_t full = bar(kFullL + s);
+        mbar_arrive_tx(full, kSub * xbox + kPBytes);
+#pragma unroll
+        for (int u = 0; u < kSub; ++u)
+          tma_load_2d(sbase + kOffX + s * kXBytes + u * xbox, &tmap_x, (kb + u) * kBK, m0, full);
+        tma_load_2d(sbase + kOffP + s * kPBytes, &tmap_w, kb * (kBK / 2), n0, full);
+      }
+      ++issued;
+    }
+    if (lane == 0) {
+      for (int j = issued - 1; j >= 0 && j >= issued - kStagesL; --j) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(bar(kFullL + j % kStagesL), (j / kStagesL) & 1) &&
+               globaltimer() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = mma_idesc_m128<F16>(ntok);
+      for (int j = 0; j < nkb; ++j) {
+        const int sb = j / kSub, sub = j % kSub, s = sb % kStagesL, t = j % kStagesB;
+        if (!mbar_wait(bar(kFullL + s), (sb / kStagesL) & 1, abort_flag)) break;
+        if (!mbar_wait(bar(kFullW + t), (j / kStagesB) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint64_t dw = sw128_kmajor_desc(sbase + kOffW + t * kWBytes);
+        const uint64_t dx = sw128_kmajor_desc(sbase + kOffX + s * kXBytes + sub * xbox);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) tc_mma(tmem, dw + 2 * k, dx + 2 * k, idesc, (j | k) != 0);
+        if (sub == kSub - 1 || j == nkb - 1) tc_commit(bar(kEmptyL + s));
+        tc_commit(bar(kEmptyW + t));
+      }
+      tc_commit(bar(kAcc));  // also the last word on any aborted run
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ dequantize
+    const int d = warp - 2;
+    const int chunk = lane & 7;
+    constexpr int kMB = MT == kF32 ? 4 : 2;
+    constexpr int kWords = MT == kF32 ? 2 : 1;
+    const int64_t groups_per_row = args.K / kBK;
+    const uint8_t* row_s[kDqIters];
+    const uint8_t* row_z[kDqIters];
+#pragma unroll
+    for (int j = 0; j < kDqIters; ++j) {
+      const int n = n0 + d * (4 * kDqIters) + j * 4 + (lane >> 3);
+      const int64_t off = static_cast<int64_t>(n) * groups_per_row * kMB;
+      row_s[j] = n < args.N ? static_cast<const uint8_t*>(args.scale) + off : nullptr;
+      row_z[j] = n < args.N ? static_cast<const uint8_t*>(args.zero) + off : nullptr;
+    }
+    uint32_t nxt_s[kDqIters], nxt_z[kDqIters], cur[kDqIters][kWords];
+    auto fetch8 = [&](int w8) {  // this lane's k-block of the 8-block window w8 of the slice
+      const int kk = kb0 + w8 * 8 + chunk;
+#pragma unroll
+      for (int j = 0; j < kDqIters; ++j) {
+        const bool in = row_s[j] != nullptr && kk < kb1;
+        nxt_s[j] = in ? meta_load<MT>(row_s[j] + static_cast<int64_t>(kk) * kMB) : 0u;
+        nxt_z[j] = in ? meta_load<MT>(row_z[j] + static_cast<int64_t>(kk) * kMB) : 0u;
+      }
+    };
+    if (nkb > 0) fetch8(0);
+    for (int j8 = 0; j8 < nkb; ++j8) {
+      const int sb = j8 / kSub, sub = j8 % kSub, s = sb % kStagesL, t = j8 % kStagesB;
+      if ((j8 & 7) == 0) {  // the window's values arrived during the previous 8 k-blocks
+#pragma unroll
+        for (int j = 0; j < kDqIters; ++j) {
+          if constexpr (kWords == 1) {
+            cur[j][0] = nxt_s[j] | (nxt_z[j] << 16);
+          } else {
+            cur[j][0] = nxt_s[j];
+            cur[j][kWords - 1] = nxt_z[j];
+          }
+        }
+        if (j8 + 8 < nkb) fetch8((j8 >> 3) + 1);
+      }
+      const int src = (lane & ~7) | (j8 & 7);
+      float sc[kDqIters], nz[kDqIters];
+#pragma unroll
+      for (int j = 0; j < kDqIters; ++j) {
+        if constexpr (kWords == 1) {
+          const uint32_t v = __shfl_sync(0xFFFFFFFFu, cur[j][0], src);
+          sc[j] = meta_f32<MT>(v & 0xFFFFu);
+          nz[j] = -meta_f32<MT>(v >> 16);
+        } else {
+          sc[j] = meta_f32<MT>(__shfl_sync(0xFFFFFFFFu, cur[j][0], src));
+          nz[j] = -meta_f32<MT>(__shfl_sync(0xFFFFFFFFu, cur[j][kWords - 1], src));
+        }
+      }
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(kFullL + s), (sb / kStagesL) & 1, abort_flag)))
+        break;
+      if (!__all_sync(0xFFFFFFFFu,
+                      mbar_wait(bar(kEmptyW + t), ((j8 / kStagesB) & 1) ^ 1, abort_flag)))
+        break;
+      const uint8_t* P = smem + kOffP + s * kPBytes;
+      uint8_t* Wt = smem + kOffW + t * kWBytes;
+      uint32_t w[kDqIters];
+#pragma unroll
+      for (int j = 0; j < kDqIters; ++j) {
+        const int row = d * (4 * kDqIters) + j * 4 + (lane >> 3);
+        w[j] = *reinterpret_cast<const uint32_t*>(P + row * 128 + sub * 32 + chunk * 4);
+      }
+#pragma unroll
+      for (int j = 0; j < kDqIters; ++j) {
+        const int row = d * (4 * kDqIters) + j * 4 + (lane >> 3);
+        *reinterpret_cast<uint4*>(Wt + row * 128 + ((chunk ^ (row & 7)) << 4)) =
+            dequant8<F16>(w[j], make_float2(nz[j], nz[j]), make_float2(sc[j], sc[j]));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kFullW + t));
+    }
+
+    // ------------------------------------------------------------ partial sums -> owners
+    // Warps 2..5 read the four TMEM lane quarters (rows 32q .. 32q+31 of the W' tile); row
+    // 16r + i goes to slot `rank` of cluster CTA r: float [kOwnRows][kTokMax] at i.
+    if (d < 4) {
+      const int quarter = warp & 3;
+      const bool ok =
+          __all_sync(0xFFFFFFFFu, mbar_wait(bar(kAcc), 0, abort_flag) && !*abort_flag);
+      tc_fence_after();
+      const int row = quarter * 32 + lane;  // W' row within the tile
+      const uint32_t owner = static_cast<uint32_t>(row / kOwnRows);
+      const uint32_t slot = sbase + kOffRed + rank * kSlotBytes +
+                            static_cast<uint32_t>(row % kOwnRows) * static_cast<uint32_t>(ntok) * 4;
+      const uint32_t dst = cluster_addr(slot, owner);
+      for (int c = 0; c < ntok; c += 16) {
+        uint32_t r[16];
+        if (ok && nkb > 0) {
+          tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + c, r);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r[i] = 0u;  // empty slice: its partial sum is 0
+        }
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+          st_cluster_v4f(dst + (c + i) * 4, __uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                         __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // every partial row has landed in its owner's slots
+  // ------------------------------------------------------------ owner: reduce and store
+  if (warp >= 2 && !*abort_flag) {
+    typedef typename std::conditional<F16, __half, __nv_bfloat16>::type T;
+    const float* red = reinterpret_cast<const float*>(smem + kOffRed);
+    const unsigned short* bias = reinterpret_cast<const unsigned short*>(args.bias);
+    const int nbase = n0 + static_cast<int>(rank) * kOwnRows;
+    // pairs (m, 2p) .. (m, 2p+1) of this CTA's 16 rows: 8 pairs per token
+    for (int idx = threadIdx.x - 64; idx < ntok * (kOwnRows / 2); idx += 32 * kDqWarps) {
+      const int m = idx / (kOwnRows / 2), pr = 2 * (idx % (kOwnRows / 2));
+      if (m0 + m >= args.M || nbase + pr >= args.N) continue;
+      float v0 = 0.0f, v1 = 0.0f;
+#pragma unroll
+      for (int src = 0; src < kS; ++src) {  // fixed order
+        v0 = __fadd_rn(v0, red[src * (kSlotBytes / 4) + pr * ntok + m]);
+        v1 = __fadd_rn(v1, red[src * (kSlotBytes / 4) + (pr + 1) * ntok + m]);
+      }
+      if (bias != nullptr) {
+        v0 = __fadd_rn(v0, F16 ? f16_bits_to_f32(bias[nbase + pr]) : bf16_bits_to_f32(bias[nbase + pr]));
+        v1 = __fadd_rn(v1, F16 ? f16_bits_to_f32(bias[nbase + pr + 1])
+                               : bf16_bits_to_f32(bias[nbase + pr + 1]));
+      }
+      *reinterpret_cast<uint32_t*>(reinterpret_cast<T*>(args.Y) +
+                                   static_cast<int64_t>(m0 + m) * args.N + nbase + pr) =
+          pack2_16<F16 ? kF16 : kBF16>(v0, v1);
+    }
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(skinny::kTmemCols)
+                 : "memory");
+  }
+}
+
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -926,52 +941,25 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// 2-D row-major tensor map: `inner` elements per row (x), `outer` rows (y), box {bx, by}.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const void* base,
+              uint64_t inner, uint64_t outer, uint32_t bx, uint32_t by,
+              CUtensorMapSwizzle swz) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * elem};
+  const cuuint32_t box[2] = {bx, by};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool F16, int MT>
 cudaError_t launch_typed(const GemmJob& job, cudaStream_t stream) {
-  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
-  if (encode == nullptr) return cudaErrorNotSupported;
-  CUtensorMap mx, mw;
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(job.K), static_cast<cuuint64_t>(job.M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(job.K) * 2};
-    const cuuint32_t box[2] = {kBK, 128};
-    const cuuint32_t estr[2] = {1, 1};
-    if (encode(&mx, F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-               const_cast<void*>(job.X), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(job.K / 2),
-                                static_cast<cuuint64_t>(job.N)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(job.K / 2)};
-    const cuuint32_t box[2] = {kBK / 2, HQQ_GEMM_2SM ? static_cast<cuuint32_t>(sm2::kRows) : kBN};
-    const cuuint32_t estr[2] = {1, 1};
-    if (encode(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(job.packed), dims,
-               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  CUtensorMap my;
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(job.N), static_cast<cuuint64_t>(job.M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(job.N) * 2};
-    const cuuint32_t box[2] = {32, 32};
-    const cuuint32_t estr[2] = {1, 1};
-    if (encode(&my, F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-               job.Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  // per device and cheap: set on every call rather than cached
-  cudaError_t e = cudaFuncSetAttribute(w4a16_gemm_kernel<F16, MT>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
-  if (e != cudaSuccess) return e;
+  const CUtensorMapDataType xdt =
+      F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   GemmArgs a;
   a.scale = job.scale;
   a.zero = job.zero;
@@ -980,31 +968,50 @@ cudaError_t launch_typed(const GemmJob& job, cudaStream_t stream) {
   a.M = static_cast<int>(job.M);
   a.N = static_cast<int>(job.N);
   a.K = static_cast<int>(job.K);
-#if HQQ_GEMM_2SM
-  e = cudaFuncSetAttribute(w4a16_gemm_2sm_kernel<F16, MT>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sm2::kSmemBytes));
-  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * static_cast<unsigned>((job.M + 511) / 512),
-                     static_cast<unsigned>((job.N + kBN - 1) / kBN));
-  cfg.blockDim = dim3(sm2::kThreads);
-  cfg.dynamicSmemBytes = sm2::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  CUtensorMap mx, mw;
+  if (job.M <= skinny::kMaxM) {
+    const int ntok = static_cast<int>(
+        (std::min<int64_t>(job.M, skinny::kTokMax) + 15) / 16 * 16);
+    if (!make_map(&mx, xdt, 2, job.X, job.K, job.M, kBK, ntok, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, job.packed, job.K / 2, job.N,
+                  kBK / 2 * skinny::kSub, skinny::kRows, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    const uint32_t smem = skinny::layout(ntok).bytes;
+    cudaError_t e = cudaFuncSetAttribute(w4a16_skinny_kernel<F16, MT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(skinny::layout(skinny::kTokMax).bytes));
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(skinny::kS * static_cast<unsigned>((job.N + skinny::kRows - 1) / skinny::kRows),
+                       static_cast<unsigned>((job.M + skinny::kTokMax - 1) / skinny::kTokMax));
+    cfg.blockDim = dim3(skinny::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    attr[0].val.clusterDim.x = skinny::kS;
+    return cudaLaunchKernelEx(&cfg, w4a16_skinny_kernel<F16, MT>, mx, mw, a, ntok);
+  }
+  CUtensorMap my;
+  if (!make_map(&mx, xdt, 2, job.X, job.K, job.M, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, job.packed, job.K / 2, job.N, kBK / 2,
+                sm2::kRows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&my, xdt, 2, job.Y, job.N, job.M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(w4a16_gemm_2sm_kernel<F16, MT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(sm2::kSmemBytes));
+  if (e != cudaSuccess) return e;
+  cfg.gridDim = dim3(2 * static_cast<unsigned>((job.M + 511) / 512),
+                     static_cast<unsigned>((job.N + kBN - 1) / kBN));
+  cfg.blockDim = dim3(sm2::kThreads);
+  cfg.dynamicSmemBytes = sm2::kSmemBytes;
+  attr[0].val.clusterDim.x = 2;
   return cudaLaunchKernelEx(&cfg, w4a16_gemm_2sm_kernel<F16, MT>, mx, mw, my, a);
-#else
-  const dim3 grid(static_cast<unsigned>((job.N + kBN - 1) / kBN),
-                  static_cast<unsigned>((job.M + kBM - 1) / kBM));
-  w4a16_gemm_kernel<F16, MT><<<grid, kThreads, kSmemBytes, stream>>>(mx, mw, my, a);
-  return cudaGetLastError();
-#endif
 }
 
 // K = 0: the sum is empty, Y[m, n] = bias[n] (or 0).

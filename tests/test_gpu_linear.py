@@ -81,7 +81,7 @@ def assert_no_timeouts():
 def test_linear_one_hot_is_bit_exact_transposed_weight():
     # N = 2·256 + 8 (ragged last tile), K = 640 (10 k-blocks: the 3-stage ring wraps 3 times),
     # M = K = 640 (ragged last M tile of 128 rows)
-    N, K = 520, 640
+    N, K = 520, 640  # M = 640 > 128: the 2-SM kernel
     codes, scale, zero, dev = make_layer(N, K, 11)
     X = torch.eye(K, dtype=torch.bfloat16)
     Y = run_linear(X, dev, N, "bf16", "bf16")
@@ -180,3 +180,40 @@ def test_linear_meta_views_with_odd_offsets():
     Y = run_linear(X, dev, N, "bf16", "bf16")
     check_against_oracle(Y, X, codes, scale, zero, N, K, "bf16")
     assert_no_timeouts()
+
+
+def test_linear_skinny_one_hot_spans_every_k_slice():
+    # M <= 128 takes the split-K kernel (8 CTAs per W' tile, each a slice of K): one-hot rows
+    # picking k = 5m + 3 reach every slice; each output is one product with 1, so Y must be
+    # the dequantized weight's columns exactly (partial sums of the other slices are +0)
+    N, K, M = 264, 1024, 100
+    codes, scale, zero, dev = make_layer(N, K, 31)
+    ks = 5 * np.arange(M) + 3
+    X = torch.zeros(M, K, dtype=torch.bfloat16)
+    X[torch.arange(M), torch.from_numpy(ks)] = 1.0
+    Y = run_linear(X, dev, N, "bf16", "bf16")
+    Wd = oracle.round_to_dtype(oracle.dequantize(codes, scale, zero, N, K, 64, 1), "bf16")
+    assert np.array_equal(Y, Wd[:, ks].T.astype(np.float64))
+    assert_no_timeouts()
+
+
+@pytest.mark.parametrize("M", [1, 7, 16, 64, 128])
+@pytest.mark.parametrize("N,K", [(4096, 4096), (11008, 4096), (4096, 11008)])
+def test_linear_skinny_llama_shapes(M, N, K):
+    codes, scale, zero, dev = make_layer(N, K, N + K + M)
+    X = make_x(M, K, 40 + M, "bf16")
+    bias = make_x(1, N, 41, "bf16")[0]
+    Y = run_linear(X, dev, N, "bf16", "bf16", bias)
+    worst, same = check_against_oracle(Y, X, codes, scale, zero, N, K, "bf16", bias)
+    assert same > 0.9, same
+    assert_no_timeouts()
+
+
+def test_linear_skinny_is_deterministic():
+    N, K, M = 1024, 2048, 33
+    codes, scale, zero, dev = make_layer(N, K, 8)
+    X = make_x(M, K, 9, "f16")
+    dev16 = make_layer(N, K, 8, "f16")[3]
+    a = run_linear(X, dev16, N, "f16", "f16")
+    b = run_linear(X, dev16, N, "f16", "f16")
+    assert np.array_equal(a, b)
