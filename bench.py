@@ -409,6 +409,32 @@ def run_linear(hqq, dev, args, tokens: int = 4096):
             profiled = {"shape_MNK": [4096, 4096, 4096],
                         "dram_bytes": t.get("dram_bytes_per_launch_4096x4096x4096"),
                         "algorithmic_bytes": 2 * 4096 * 4096 * 2 + 4096 * 4096 // 2 + 4096 * 64 * 4}
+    # decode-sized batch: the same layers at 16 tokens take the split-K kernel; weight-read
+    # bound (0.5 B of codes + 4/64 B of bf16 scale/zero per weight from HBM)
+    dec_tokens = 16
+    dec = []
+    for m, X, pk, sc, zr, Y, Wd in layers:
+        Xd = X[:dec_tokens].contiguous()
+        Yd = torch.empty(dec_tokens, m.rows, dtype=torch.bfloat16, device=dev)
+        dec.append((m, Xd, pk, sc, zr, Yd))
+    for _ in range(args.warmup):
+        for m, Xd, pk, sc, zr, Yd in dec:
+            hqq.hqq_linear(Xd, pk, sc, zr, m.rows, Y=Yd, stream=stream)
+    dec_ms = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in dec]
+        for (a, b), (m, Xd, pk, sc, zr, Yd) in zip(evs, dec):
+            a.record(stream)
+            hqq.hqq_linear(Xd, pk, sc, zr, m.rows, Y=Yd, stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        dec_ms.append(sum(a.elapsed_time(b) for a, b in evs))
+    ms_dec = statistics.median(dec_ms)
+    wbytes = sum(m.rows * m.cols * (0.5 + 4 / 64) for m, *_ in dec)
+    hbm = peaks()["hbm_gbs"]
+    dec_gbs = wbytes / (ms_dec * 1e-3) / 1e9
     return {
         "metric": "fused 4-bit linear TFLOP/s", "value": round(tf, 1), "unit": "TFLOP/s",
         "workload": f"Llama-7B block linear layers, {tokens} tokens, bf16 activations, "
@@ -423,8 +449,16 @@ def run_linear(hqq, dev, args, tokens: int = 4096):
                      "algorithmic": "2*M*N*K flops per launch",
                      "peak_source": f"bf16 dense, {source} (burst: the kernel is timed alone)"},
         "l2": "flushed before every step",
+        "decode_16_tokens": {
+            "kernel": "w4a16_skinny_kernel (split-K over a 4-CTA cluster)",
+            "ms_per_step": round(ms_dec, 4), "launches_per_step": len(dec),
+            "tflops": round(sum(2.0 * dec_tokens * m.rows * m.cols for m, *_ in dec)
+                            / (ms_dec * 1e-3) / 1e12, 2),
+            "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(dec_gbs / hbm, 4),
+                         "algorithmic": "0.5625 B of packed codes + scale/zero per weight"}},
         "wait_timeouts": hqq.hqq_wait_timeouts(),
-        "gpu_launches": len(layers) * args.steps,
+        "gpu_launches": 2 * len(layers) * args.steps,
     }
 
 
