@@ -692,11 +692,12 @@ def probe_hbm(gib: float = 1.0):
     return res
 
 
-def single_linear(reps: int = 10):
-    """One 4096 x 4096 x 4096 hqq_linear launch (bf16, 4-bit g64): the ncu profiling case."""
+def single_linear(reps: int = 10, M: int = 4096):
+    """One 4096 x 4096 hqq_linear launch with M tokens (bf16, 4-bit g64): the ncu profiling
+    cases (M = 4096: the 2-SM kernel; M = 16: the split-K kernel)."""
     import calibration_free_weight_hqq_b200 as hqq
     from calibration_free_weight_hqq_b200 import synthetic
-    M = N = K = 4096
+    N = K = 4096
     W = synthetic.weight(N, K, seed=11, dtype=torch.bfloat16, device="cuda")
     pk, s, z = hqq.hqq_quantize(W, 4, 64, 1)
     X = synthetic.activations(M, K, seed=12, device="cuda")
@@ -765,9 +766,9 @@ def main():
                     help="measure the lg2/ex2 issue rate behind the roofline peak and exit")
     ap.add_argument("--probe-hbm", action="store_true",
                     help="measure HBM read-only, write-only and copy bandwidth and exit")
-    ap.add_argument("--single", choices=["quantize", "dequantize", "linear"],
-                    help="time one [16384,8192] matrix, or one 4096^3 linear layer (the "
-                         "profiling cases), and exit")
+    ap.add_argument("--single", choices=["quantize", "dequantize", "linear", "decode"],
+                    help="time one [16384,8192] matrix, one 4096^3 linear layer, or one "
+                         "4096x4096 layer at 16 tokens (the profiling cases), and exit")
     args = ap.parse_args()
     if args.probe_sfu:
         print(json.dumps(probe_sfu()), flush=True)
@@ -776,8 +777,10 @@ def main():
         print(json.dumps(probe_hbm()), flush=True)
         return
     if args.single:
-        print(json.dumps(single_linear() if args.single == "linear" else single(args.single)),
-              flush=True)
+        if args.single in ("linear", "decode"):
+            print(json.dumps(single_linear(M=4096 if args.single == "linear" else 16)), flush=True)
+        else:
+            print(json.dumps(single(args.single)), flush=True)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
