@@ -160,8 +160,8 @@ static hqq_status quantize_impl(const void* W, int64_t rows, int64_t cols, const
   j.packed = reinterpret_cast<uint8_t*>(Wq_packed);
   j.scale = qs ? static_cast<void*>(ws_scale) : scale;
   j.zero = qz ? static_cast<void*>(ws_zero) : zero;
-  j.scale_dtype = qs ? hqqk::kF32 : prm.meta_dtype;
-  j.zero_dtype = qz ? hqqk::kF32 : prm.meta_dtype;
+  j.scale_dtype = qs ? static_cast<int>(hqqk::kF32) : static_cast<int>(prm.meta_dtype);
+  j.zero_dtype = qz ? static_cast<int>(hqqk::kF32) : static_cast<int>(prm.meta_dtype);
   j.flags = prm.flags;
   if ((st = cuda_status(hqqk::launch_quantize(j, stream))) != HQQ_OK) return st;
   if (qs) {

@@ -13,7 +13,8 @@ import torch
 import calibration_free_weight_hqq_b200 as hqq
 from calibration_free_weight_hqq_b200 import synthetic, workloads
 import oracle
-from parity import compare, group_view, sample_groups, unpack_groups
+from parity import (compare, dequant_parity, exact_grid_weights, group_view, np_unpack,
+                    sample_groups, unpack_groups)
 
 pytestmark = pytest.mark.gpu
 
@@ -134,7 +135,7 @@ def test_constant_groups():
     pk, s, z = hqq.hqq_quantize(W, 4, 64, 1)
     assert torch.all(s[5] == 1) and torch.all(z[5] == -0.25) and torch.all(z[17] == 0)
     assert s[9, 0] == 1 and z[9, 0] == 1.0
-    codes = oracle.unpack(pk.cpu().numpy(), W.numel(), 4).reshape(1024, 1024)
+    codes = np_unpack(pk.cpu().numpy(), W.numel(), 4).reshape(1024, 1024)
     assert np.all(codes[5] == 0) and np.all(codes[17] == 0) and np.all(codes[9, :64] == 0)
 
 
@@ -194,15 +195,45 @@ def test_stored_meta_dtype_is_rounded_once(dtype):
     assert (o_z != z.reshape(-1).cpu()).sum().item() <= 1e-4 * oz.size
 
 
-@pytest.mark.parametrize("out_dtype", [torch.float16, torch.bfloat16, torch.float32])
-def test_dequantize_out_dtypes_bit_exact(out_dtype):
-    W = synthetic.weight(128, 512, seed=18, dtype=torch.bfloat16, device=DEV)
-    pk, s, z = hqq.hqq_quantize(W, 4, 64, 1)
-    D = hqq.hqq_dequantize(pk, s, z, 128, 512, 4, 64, 1, out_dtype=out_dtype)
-    codes = oracle.unpack(pk.cpu().numpy(), 128 * 512, 4)
-    ref = oracle.dequantize(codes, s.float().reshape(-1).cpu().numpy(),
-                            z.float().reshape(-1).cpu().numpy(), 128, 512, 64, 1)
-    assert torch.equal(torch.from_numpy(ref).to(out_dtype), D.cpu())
+@pytest.mark.parametrize("nbits,G,axis", [(8, 8, 1), (4, 64, 1), (4, 128, 0), (3, 64, 1),
+                                          (3, 32, 0), (2, 16, 1), (2, 16, 0), (1, 32, 1),
+                                          (1, 256, 0), (4, 256, 1)])
+def test_packing_bit_exact_on_exact_grids(nbits, G, axis):
+    # codes, step and zero known by construction (not from either implementation): the GPU
+    # quantizer must reproduce them and pack them exactly as the oracle's packer does
+    rows, cols = (4 * G, 320) if axis == 0 else (96, 5 * G)
+    W, q, step, z = exact_grid_weights(rows, cols, nbits, G, axis, seed=nbits * 1000 + G)
+    params = hqq.make_params(nbits, G, axis, w_dtype=torch.bfloat16, meta_dtype=torch.float32)
+    out = hqq.hqq_quantize_ex(W, params)
+    torch.cuda.synchronize()
+    assert np.array_equal(out["Wq_packed"].cpu().numpy(), oracle.pack(q, nbits))
+    assert np.array_equal(out["scale"].reshape(-1).cpu().numpy(), step)
+    assert np.array_equal(out["zero"].reshape(-1).cpu().numpy(), z)
+
+
+@pytest.mark.parametrize("nbits,G,axis", [(8, 32, 1), (4, 64, 1), (4, 64, 0), (3, 64, 1),
+                                          (3, 16, 0), (2, 16, 1), (1, 32, 1), (1, 8, 0)])
+@pytest.mark.parametrize("out_dtype", ["f16", "bf16", "f32"])
+def test_dequantize_bit_exact(nbits, G, axis, out_dtype):
+    rows, cols = (3 * G + G, 200) if axis == 0 else (37, 12 * G)
+    for meta in ("f32", "bf16", "f16"):
+        dequant_parity(rows, cols, nbits, G, axis, out_dtype, meta_dtype=meta,
+                       seed=nbits * 97 + G + axis)
+
+
+@pytest.mark.parametrize("nbits,G,axis", [(4, 64, 1), (3, 64, 1), (2, 16, 0), (1, 32, 1)])
+def test_dequantize_bit_exact_second_level(nbits, G, axis):
+    rows, cols = (8 * G, 192) if axis == 0 else (64, 40 * G)
+    for mg in (128, 100):
+        dequant_parity(rows, cols, nbits, G, axis, "bf16", quant_meta=True, meta_group=mg,
+                       seed=nbits + mg)
+
+
+@pytest.mark.parametrize("rows,cols", [(16384, 8192), (4096, 11008)])
+def test_dequantize_bit_exact_bench_layout(rows, cols):
+    # 4-bit, group 64, axis 1, bf16 meta and output: the layout of the bench step (its
+    # dedicated kernel), on full-size matrices
+    dequant_parity(rows, cols, 4, 64, 1, "bf16", meta_dtype="bf16", seed=rows)
 
 
 def test_quantize_meta_standalone():
@@ -243,7 +274,7 @@ def test_more_than_2_pow_32_elements():
     oc, os_, oz = oracle.quantize(Wg, 4, G, 1, 20, 0.7, 10.0, 1.01, nthreads=8)
     per = G * 4 // 8
     pkg = pk.reshape(ng, per)[ids_t].cpu().numpy()
-    gc = oracle.unpack(pkg.ravel(), ids.size * G, 4).reshape(-1, G)
+    gc = np_unpack(pkg.ravel(), ids.size * G, 4).reshape(-1, G)
     assert np.count_nonzero(gc != oc) <= 1e-3 * gc.size
     assert torch.equal(s.reshape(-1)[ids_t].cpu(), torch.from_numpy(os_).to(torch.bfloat16))
     del W
