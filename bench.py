@@ -717,6 +717,60 @@ def single_linear(reps: int = 10, M: int = 4096):
             "wait_timeouts": hqq.hqq_wait_timeouts()}
 
 
+def configs_table(reps: int = 3):
+    """Quantize and dequantize throughput of the four smaller workloads of the pages'
+    configurations (the fifth, the whole model, is the headline), one line per configuration:
+    solver Gweights/s and its MUFU fraction, dequantizer algorithmic GB/s and its HBM fraction.
+    Each matrix is timed with CUDA events over `reps` launches after one warm-up."""
+    import calibration_free_weight_hqq_b200 as hqq
+    from calibration_free_weight_hqq_b200 import workloads
+    pk = peaks()
+    mufu_peak = MUFU_PER_CLK_PER_SM * N_SM * pk["sm_max_mhz"] * 1e6
+    out = []
+    for wl in (workloads.single_fp16(), workloads.llama7b_block_4b(),
+               workloads.llama7b_block_2b_axis0(), workloads.mlp70b_mixed()):
+        q_ms = d_ms = 0.0
+        dq_bytes = 0
+        for m in wl.matrices:
+            W = workloads.make_weight(m, "cuda")
+            params = hqq.make_params(m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0,
+                                     m.kappa, w_dtype=m.dtype, quant_scale=m.quant_meta,
+                                     quant_zero=m.quant_meta,
+                                     meta_group_size=m.meta_group_size)
+            need = hqq.hqq_workspace_bytes(m.rows, m.cols, params)
+            ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda") if need else None
+            q = hqq.hqq_quantize_ex(W, params, workspace=ws)
+            D = torch.empty_like(W)
+
+            def timed(fn):
+                fn()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(reps):
+                    fn()
+                e1.record()
+                torch.cuda.synchronize()
+                return e0.elapsed_time(e1) / reps
+
+            q_ms += timed(lambda: hqq.hqq_quantize_ex(W, params, out=q, workspace=ws))
+            d_ms += timed(lambda: hqq.hqq_dequantize_ex(q, m.rows, m.cols, params, out_dtype=m.dtype,
+                                                        out=D))
+            ng = m.numel // m.group_size
+            meta_b = 2 * ng * (1 if m.quant_meta else 2)
+            dq_bytes += hqq.hqq_packed_bytes(m.rows, m.cols, m.nbits) + meta_b + 2 * m.numel
+            del W, D, q, ws
+        n = wl.weights
+        mufu = 2 * (wl.matrices[0].iters + 1) * n / (q_ms * 1e-3)
+        gbs = dq_bytes / (d_ms * 1e-3) / 1e9
+        out.append({"workload": wl.name, "weights": n,
+                    "quantize_ms": round(q_ms, 3), "quantize_Gweights_per_s": round(n / q_ms / 1e6, 2),
+                    "quantize_mufu_frac": round(mufu / mufu_peak, 4),
+                    "dequantize_ms": round(d_ms, 4), "dequantize_GB_per_s": round(gbs, 1),
+                    "dequantize_hbm_frac": round(gbs / pk["hbm_gbs"], 4)})
+    return out
+
+
 def single(kind: str, reps: int = 10):
     """One [16384, 8192] bf16 matrix (134M weights, 268 MB: larger than L2), 4-bit g64:
     time `reps` solver or dequantize launches after warm-up (the small case the ncu
@@ -766,6 +820,8 @@ def main():
                     help="measure the lg2/ex2 issue rate behind the roofline peak and exit")
     ap.add_argument("--probe-hbm", action="store_true",
                     help="measure HBM read-only, write-only and copy bandwidth and exit")
+    ap.add_argument("--configs", action="store_true",
+                    help="quantize/dequantize throughput of the four smaller configurations")
     ap.add_argument("--single", choices=["quantize", "dequantize", "linear", "decode"],
                     help="time one [16384,8192] matrix, one 4096^3 linear layer, or one "
                          "4096x4096 layer at 16 tokens (the profiling cases), and exit")
@@ -775,6 +831,10 @@ def main():
         return
     if args.probe_hbm:
         print(json.dumps(probe_hbm()), flush=True)
+        return
+    if args.configs:
+        for line in configs_table():
+            print(json.dumps(line), flush=True)
         return
     if args.single:
         if args.single in ("linear", "decode"):

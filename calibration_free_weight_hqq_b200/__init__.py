@@ -204,9 +204,11 @@ def hqq_quantize(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: in
     return Wq_packed, scale, zero
 
 
-def hqq_quantize_ex(W: torch.Tensor, params: HQQParams, *, stream=None, workspace=None):
+def hqq_quantize_ex(W: torch.Tensor, params: HQQParams, *, stream=None, workspace=None,
+                    out: Optional[dict] = None):
     """Full parameter set (second-level 8-bit scale/zero). Returns a dict with Wq_packed,
-    scale, zero (uint8 codes when quantized) and scale_mm / zero_mm (fp32 [runs, 2])."""
+    scale, zero (uint8 codes when quantized) and scale_mm / zero_mm (fp32 [runs, 2]); `out`,
+    a dict of that form from an earlier call, is written in place."""
     rows, cols = W.shape
     wp = _cuda(W, "W")
     dev = W.device
@@ -216,7 +218,7 @@ def hqq_quantize_ex(W: torch.Tensor, params: HQQParams, *, stream=None, workspac
     ms = _meta_shape(rows, cols, params.group_size, params.axis)
     mdt = _DT_TORCH[params.meta_dtype]
     runs = max(hqq_num_meta_groups(ng, params.meta_group_size), 0)
-    out = {
+    out = out if out is not None else {
         "Wq_packed": torch.empty(hqq_packed_bytes(rows, cols, params.nbits), dtype=torch.uint8,
                                  device=dev),
         "scale": torch.empty(ms, dtype=torch.uint8 if params.quant_scale else mdt, device=dev),

@@ -345,6 +345,75 @@ __global__ void __launch_bounds__(kDBlock)
   }
 }
 
+// axis=0 with small groups (G*NB <= 64 bits) and a 16-bit output: a group is one column's G
+// consecutive rows and its G*NB bits are contiguous in the stream, so a lane takes 8 adjacent
+// columns of one row block, loads their 8 groups' codes (8*G*NB/8 bytes, one to four 16-byte
+// loads) and meta once, and writes one 16-byte run per row of the block: a warp (256 columns)
+// writes 512 contiguous bytes per row. Work unit = (row block, 256 columns), one per warp.
+constexpr int kD0Cols = 256;  // columns per warp unit
+
+template <int NB, int G, int OUT_DT, int MAXB>
+__global__ void __launch_bounds__(kDBlock) dequant_axis0_cols_kernel(
+    const __grid_constant__ DBatch<MAXB> batch) {
+  constexpr int kBg = G * NB / 8;  // bytes per group: 1, 2, 4 or 8
+  constexpr int kWords = 2 * kBg;  // 8 groups
+  static_assert(kBg == 1 || kBg == 2 || kBg == 4 || kBg == 8, "group bytes");
+  const int64_t total = batch.tile_start[batch.n];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+    int64_t local;
+    const DArgs a = batch_args(batch, t, &local);
+    const int64_t cunits = (a.cols + kD0Cols - 1) / kD0Cols;
+    const int64_t unit = local * (kDBlock / 32) + warp;
+    const int64_t rb = unit / cunits;
+    if (rb >= a.rows / G) continue;
+    const int64_t c0 = (unit - rb * cunits) * kD0Cols + lane * 8;
+    if (c0 >= a.cols) continue;  // cols % 8 == 0 on this path: 8 columns are all in or out
+    const int64_t g0 = rb * a.cols + c0;
+    const uint8_t* src = a.packed + g0 * kBg;  // 8 consecutive groups, 8*kBg-byte aligned
+    uint32_t wd[kWords];
+    if constexpr (kBg == 1) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
+      wd[0] = v.x;
+      wd[1] = v.y;
+    } else {
+#pragma unroll
+      for (int q = 0; q < kWords / 4; ++q) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + q);
+        wd[4 * q] = v.x;
+        wd[4 * q + 1] = v.y;
+        wd[4 * q + 2] = v.z;
+        wd[4 * q + 3] = v.w;
+      }
+    }
+    // group i's G*NB bits (stream bits i*G*NB ..) in one 64-bit register, compile-time indices
+    uint64_t gw[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if constexpr (kBg == 8)
+        gw[i] = static_cast<uint64_t>(wd[2 * i]) | (static_cast<uint64_t>(wd[2 * i + 1]) << 32);
+      else
+        gw[i] = (wd[i * kBg / 4] >> (8 * ((i * kBg) % 4))) & ((1ull << (8 * kBg)) - 1ull);
+    }
+    float sc[8], nz[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      sc[i] = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g0 + i);
+      nz[i] = -meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g0 + i);
+    }
+#pragma unroll 4
+    for (int j = 0; j < G; ++j) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t q = static_cast<uint32_t>(gw[i] >> (j * NB)) & ((1u << NB) - 1u);
+        v[i] = __fmul_rn(__fadd_rn(u2f_small(q), nz[i]), sc[i]);
+      }
+      store8<OUT_DT>(a.out, (rb * G + j) * a.cols + c0, v);
+    }
+  }
+}
+
 // SMs x resident blocks per SM of `kernel` on the current device (host-side query).
 template <typename K>
 static cudaError_t resident_blocks(K kernel, int* out) {
@@ -392,6 +461,32 @@ static void fill_dbatch(const DequantJob* jobs, int n, int64_t tile_elems, DBatc
   b->n = k;
 }
 
+// The axis-0 column kernel for groups of G (G >= 8; G * NB <= 64 bits); tiles count its warp
+// units (row block, 256 columns), kDBlock / 32 per block.
+template <int NB, int G, int OUT_DT, int MAXB>
+static cudaError_t launch_axis0_cols(const DequantJob* jobs, int n, cudaStream_t st) {
+  if constexpr (G < 8) {
+    return cudaErrorNotSupported;
+  } else {
+    DBatch<MAXB> b;
+    fill_dbatch<MAXB>(jobs, n, kDTile0, &b);
+    int64_t tiles = 0;
+    for (int k = 0; k < b.n; ++k) {
+      b.tile_start[k] = tiles;
+      const int64_t units = (b.rows[k] / G) * ((b.cols[k] + kD0Cols - 1) / kD0Cols);
+      tiles += (units + kDBlock / 32 - 1) / (kDBlock / 32);
+    }
+    b.tile_start[b.n] = tiles;
+    if (tiles == 0) return cudaSuccess;
+    int resident = 0;
+    const cudaError_t e = resident_blocks(dequant_axis0_cols_kernel<NB, G, OUT_DT, MAXB>, &resident);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = tiles < resident ? tiles : resident;
+    dequant_axis0_cols_kernel<NB, G, OUT_DT, MAXB><<<(unsigned)blocks, kDBlock, 0, st>>>(b);
+    return cudaGetLastError();
+  }
+}
+
 template <int NB, int OUT_DT, int MAXB>
 static cudaError_t launch_nb_dt(const DequantJob* jobs, int n, cudaStream_t st) {
   DBatch<MAXB> b;
@@ -420,6 +515,19 @@ static cudaError_t launch_nb_dt(const DequantJob* jobs, int n, cudaStream_t st) 
     const int64_t blocks = tiles < resident ? tiles : resident;
     dequant_axis1_kernel<NB, OUT_DT, MAXB><<<(unsigned)blocks, kDBlock, 0, st>>>(b);
   } else {
+    if constexpr (OUT_DT != kF32 && NB != 3) {
+      bool cols8 = true;
+      for (int i = 0; i < n; ++i) cols8 = cols8 && jobs[i].cols % 8 == 0;
+      const int G = jobs[0].group_size;
+      cudaError_t e = cudaErrorNotSupported;
+      if (cols8) {
+        if (NB * G == 16) e = launch_axis0_cols<NB, 16 / NB, OUT_DT, MAXB>(jobs, n, st);
+        else if (NB * G == 32) e = launch_axis0_cols<NB, 32 / NB, OUT_DT, MAXB>(jobs, n, st);
+        else if (NB * G == 64) e = launch_axis0_cols<NB, 64 / NB, OUT_DT, MAXB>(jobs, n, st);
+        else if (NB * G == 8) e = launch_axis0_cols<NB, 8 / NB, OUT_DT, MAXB>(jobs, n, st);
+      }
+      if (e != cudaErrorNotSupported) return e;
+    }
     fill_dbatch<MAXB>(jobs, n, kDTile0, &b);
     const int64_t tiles = b.tile_start[b.n];
     if (tiles == 0) return cudaSuccess;

@@ -212,9 +212,12 @@ def test_packing_bit_exact_on_exact_grids(nbits, G, axis):
 
 
 @pytest.mark.parametrize("nbits,G,axis", [(8, 32, 1), (4, 64, 1), (4, 64, 0), (3, 64, 1),
-                                          (3, 16, 0), (2, 16, 1), (1, 32, 1), (1, 8, 0)])
+                                          (3, 16, 0), (2, 16, 1), (1, 32, 1), (1, 8, 0),
+                                          (2, 16, 0), (2, 32, 0), (4, 16, 0), (8, 8, 0),
+                                          (1, 64, 0)])
 @pytest.mark.parametrize("out_dtype", ["f16", "bf16", "f32"])
 def test_dequantize_bit_exact(nbits, G, axis, out_dtype):
+    # axis 0 with 200 columns: the last 256-column unit of the column kernel is partial
     rows, cols = (3 * G + G, 200) if axis == 0 else (37, 12 * G)
     for meta in ("f32", "bf16", "f16"):
         dequant_parity(rows, cols, nbits, G, axis, out_dtype, meta_dtype=meta,
@@ -279,3 +282,10 @@ def test_more_than_2_pow_32_elements():
     assert torch.equal(s.reshape(-1)[ids_t].cpu(), torch.from_numpy(os_).to(torch.bfloat16))
     del W
     torch.cuda.empty_cache()
+
+
+def test_dequantize_axis0_column_kernel_large_and_ragged():
+    # the config-3 layout (2-bit, group 16, axis 0) at a Llama shape, and a width that is not a
+    # multiple of 8 (the element-wise kernel)
+    dequant_parity(11008, 4096, 2, 16, 0, "bf16", meta_dtype="bf16", seed=3)
+    dequant_parity(64, 4100, 2, 16, 0, "bf16", meta_dtype="bf16", seed=4)
