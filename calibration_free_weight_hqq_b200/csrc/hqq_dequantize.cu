@@ -6,12 +6,15 @@
 // With the second level ("HQQ tutorial" (devpress.csdn.net) §3.3, quant_scale/quant_zero),
 // scale_g (zero_g) is first rebuilt in fp32 as (code - zero2)*step2 of its run.
 //
-// Layout on B200: HBM-bound (about 2.5 bytes per weight at 4 bits). A thread writes chunks of
-// 8 consecutive outputs with one 16-byte streaming store each (two for fp32), so a warp stores
-// 512 contiguous bytes per instruction; for axis=1 the 8 codes come from one 1..8-byte load
-// (or two 32-bit words for 3 bits) with one scale/zero pair. Codes become floats through the
-// 2^23 mantissa trick and group indices through shifts, keeping the slow conversion/XU pipe
-// and 64-bit division out of the per-element work.
+// Layout on B200: HBM-bound (about 2.5 bytes per weight at 4 bits). A lane writes chunks of 8
+// consecutive outputs with one 16-byte streaming store each (two for fp32), so a warp stores
+// 512 contiguous bytes per instruction, and a warp issues the loads of several chunks before
+// converting any. Codes become floats through the 2^23 mantissa trick and group indices
+// through shifts, keeping the slow conversion/XU pipe and 64-bit division out of the
+// per-element work. Kernels: dequant4_axis1_kernel (4 bits, plain meta, 16-bit output: the
+// bench layout), dequant_axis1_kernel (every other axis-1 layout), dequant_axis0_cols_kernel
+// (axis 0, groups of at most 64 bits, width a multiple of 8) and dequant_axis0_kernel (the
+// remaining axis-0 layouts, element by element).
 #include "hqq_device.cuh"
 #include "hqq_kernels.h"
 
@@ -19,28 +22,10 @@ namespace hqqk {
 
 constexpr int kDBlock = 256;
 
-// Tuning knobs (compile-time): chunks of 8 elements in flight per thread, streaming
-// (evict-first) output stores, minimum resident blocks per SM.
-#ifndef HQQ_DQ_CHUNKS
-#define HQQ_DQ_CHUNKS 2
-#endif
-#ifndef HQQ_DQ_STCS
-#define HQQ_DQ_STCS 1
-#endif
-#ifndef HQQ_DQ_MINB
-#define HQQ_DQ_MINB 8
-#endif
-#ifndef HQQ_DQ_PREFETCH
-#define HQQ_DQ_PREFETCH 1
-#endif
-
+// Output stores are streaming (evict-first): the result is not read back by this pass.
 template <typename T>
 __device__ __forceinline__ void st_out(T* p, const T& v) {
-#if HQQ_DQ_STCS
   __stcs(p, v);
-#else
-  *p = v;
-#endif
 }
 
 struct DArgs {
@@ -182,84 +167,47 @@ __device__ __forceinline__ uint32_t code_in(uint64_t raw, int off, int i) {
   }
 }
 
-// axis=1: 8 consecutive elements share one group and have consecutive codes. Grid-stride
-// over chunks of 8 elements at full occupancy; each pass a thread loads kDChunks chunks
-// (kDBlock chunks apart, so a warp's accesses of one chunk index are contiguous) before it
-// computes and stores any, keeping that many loads in flight.
-constexpr int kDChunks = HQQ_DQ_CHUNKS;
+// axis=1: 8 consecutive elements share one group and have consecutive codes. A warp covers
+// 256 consecutive elements per chunk (lane l: elements 8l .. 8l+7: their codes in one load of
+// 1..8 bytes, or two 32-bit words for 3 bits, their group's meta, one 16- or 32-byte store),
+// kD1Unroll chunks per warp per tile with every load of the tile issued before any conversion.
+// Any nbits, plain or second-level meta, any output type.
+constexpr int kD1Unroll = 4;
+constexpr int64_t kDTile1 = (int64_t)kDBlock * 8 * kD1Unroll;
 
-// Elements per tile of the axis-1 kernel (kDChunks chunks of 8 per thread).
-constexpr int64_t kDTile1 = (int64_t)kDBlock * kDChunks * 8;
-
-// One round of a thread's work: kDChunks chunks of 8 elements of one tile, loaded.
-template <int NB>
-struct DRound {
-  const uint8_t* packed;
-  void* out;
-  int64_t c0, n_chunks, n;
-  uint64_t raw[kDChunks];
-  int off[kDChunks];
-  float sc[kDChunks], zr[kDChunks];
-};
-
-template <int NB, int MAXB>
-__device__ __forceinline__ void load_round(const DBatch<MAXB>& batch, int64_t t, DRound<NB>& r) {
-  int64_t local;
-  const DArgs a = batch_args(batch, t, &local);
-  r.packed = a.packed;
-  r.out = a.out;
-  r.n = a.n;
-  r.n_chunks = a.n >> 3;
-  r.c0 = local * kDBlock * kDChunks + threadIdx.x;
-#pragma unroll
-  for (int i = 0; i < kDChunks; ++i) {
-    const int64_t c = r.c0 + (int64_t)i * kDBlock;
-    if (c < r.n_chunks) {
-      r.raw[i] = codes8_raw<NB>(a.packed, c << 3, a.n, r.off[i]);
-      const int64_t g = (c << 3) >> a.log2_group;
-      r.sc[i] = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g);
-      r.zr[i] = meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g);
-    }
-  }
-}
-
-template <int NB, int OUT_DT>
-__device__ __forceinline__ void finish_round(const DRound<NB>& r) {
-#pragma unroll
-  for (int i = 0; i < kDChunks; ++i) {
-    const int64_t c = r.c0 + (int64_t)i * kDBlock;
-    if (c < r.n_chunks) {
-      float v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        v[j] = __fmul_rn(__fsub_rn(u2f_small(code_in<NB>(r.raw[i], r.off[i], j)), r.zr[i]), r.sc[i]);
-      store8<OUT_DT>(r.out, c << 3, v);  // n and G are multiples of 8 on this path
-    }
-  }
-}
-
-// Grid-stride over tiles; the loads of a thread's next round are issued before the current
-// round is converted and stored, so load latency overlaps the stores instead of following
-// them.
 template <int NB, int OUT_DT, int MAXB>
-__global__ void __launch_bounds__(kDBlock, HQQ_DQ_MINB)
-    dequant_axis1_kernel(const __grid_constant__ DBatch<MAXB> batch) {
+__global__ void __launch_bounds__(kDBlock) dequant_axis1_kernel(
+    const __grid_constant__ DBatch<MAXB> batch) {
   const int64_t total = batch.tile_start[batch.n];
-  int64_t t = blockIdx.x;
-  if (t >= total) return;
-  DRound<NB> cur;
-  load_round<NB>(batch, t, cur);
-  for (; t < total; t += gridDim.x) {
-#if HQQ_DQ_PREFETCH
-    DRound<NB> nxt;
-    const bool more = t + gridDim.x < total;
-    if (more) load_round<NB>(batch, t + gridDim.x, nxt);
-    finish_round<NB, OUT_DT>(cur);
-    if (more) cur = nxt;
-#else
-    finish_round<NB, OUT_DT>(cur);
-    if (t + gridDim.x < total) load_round<NB>(batch, t + gridDim.x, cur);
-#endif
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+    int64_t local;
+    const DArgs a = batch_args(batch, t, &local);
+    const int64_t base = local * kDTile1 + (int64_t)warp * (kD1Unroll * 256) + lane * 8;
+    uint64_t raw[kD1Unroll];
+    int off[kD1Unroll];
+    float sc[kD1Unroll], zr[kD1Unroll];
+#pragma unroll
+    for (int u = 0; u < kD1Unroll; ++u) {
+      const int64_t i = base + u * 256;
+      if (i < a.n) {  // n and G are multiples of 8: a lane's 8 elements share one group
+        raw[u] = codes8_raw<NB>(a.packed, i, a.n, off[u]);
+        const int64_t g = i >> a.log2_group;
+        sc[u] = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g);
+        zr[u] = meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kD1Unroll; ++u) {
+      const int64_t i = base + u * 256;
+      if (i < a.n) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          v[j] = __fmul_rn(__fsub_rn(u2f_small(code_in<NB>(raw[u], off[u], j)), zr[u]), sc[u]);
+        store8<OUT_DT>(a.out, i, v);
+      }
+    }
   }
 }
 
