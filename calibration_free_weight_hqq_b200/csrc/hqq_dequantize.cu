@@ -35,6 +35,7 @@ struct DArgs {
   const float* scale_mm;
   const float* zero_mm;
   int meta_group_size, meta_dtype;
+  int log2_meta_group;    // log2(meta_group_size) when it is a power of two, else -1
   int64_t rows, cols, n;  // n = rows*cols
   int group_size, log2_group;
   void* out;
@@ -84,14 +85,18 @@ __device__ __forceinline__ float u2f_small(uint32_t q) {
   return __fsub_rn(__uint_as_float(q | 0x4B000000u), 8388608.0f);
 }
 
-__device__ __forceinline__ float meta_value(const void* p, const float* mm, int mdt, int mgs,
+// Scale or zero of group g: stored directly, or as an 8-bit code of the second level
+// decoded with its run's (step, zero) pair. The run index is a shift for power-of-two runs
+// (a 64-bit division otherwise).
+__device__ __forceinline__ float meta_value(const DArgs& a, const void* p, const float* mm,
                                             int64_t g) {
   if (mm) {
-    const int64_t run = g / mgs;
-    const float q = u2f_small(reinterpret_cast<const uint8_t*>(p)[g]);
-    return __fmul_rn(__fsub_rn(q, mm[2 * run + 1]), mm[2 * run]);
+    const int64_t run = a.log2_meta_group >= 0 ? g >> a.log2_meta_group : g / a.meta_group_size;
+    const float q = u2f_small(__ldg(reinterpret_cast<const uint8_t*>(p) + g));
+    const float2 sz = __ldg(reinterpret_cast<const float2*>(mm) + run);
+    return __fmul_rn(__fsub_rn(q, sz.y), sz.x);
   }
-  return load_meta(p, mdt, g);
+  return load_meta(p, a.meta_dtype, g);
 }
 
 // Code with stream index k (layout of the header).
@@ -193,8 +198,8 @@ __global__ void __launch_bounds__(kDBlock) dequant_axis1_kernel(
       if (i < a.n) {  // n and G are multiples of 8: a lane's 8 elements share one group
         raw[u] = codes8_raw<NB>(a.packed, i, a.n, off[u]);
         const int64_t g = i >> a.log2_group;
-        sc[u] = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g);
-        zr[u] = meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g);
+        sc[u] = meta_value(a, a.scale, a.scale_mm, g);
+        zr[u] = meta_value(a, a.zero, a.zero_mm, g);
       }
     }
 #pragma unroll
@@ -272,8 +277,8 @@ __global__ void __launch_bounds__(kDBlock)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int64_t g = rb * a.cols + c0 + i;
-      const float sc = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g);
-      const float zr = meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g);
+      const float sc = meta_value(a, a.scale, a.scale_mm, g);
+      const float zr = meta_value(a, a.zero, a.zero_mm, g);
       const float q = u2f_small(code_at<NB>(a.packed, (g << a.log2_group) + j));
       v[i] = __fmul_rn(__fsub_rn(q, zr), sc);
     }
@@ -286,8 +291,8 @@ __global__ void __launch_bounds__(kDBlock)
     const int64_t rb = r / G;
     const int j = (int)(r - rb * G);
     const int64_t g = rb * a.cols + c;
-    const float sc = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g);
-    const float zr = meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g);
+    const float sc = meta_value(a, a.scale, a.scale_mm, g);
+    const float zr = meta_value(a, a.zero, a.zero_mm, g);
     const float q = u2f_small(code_at<NB>(a.packed, g * G + j));
     store1<OUT_DT>(a.out, k, __fmul_rn(__fsub_rn(q, zr), sc));
   }
@@ -346,8 +351,8 @@ __global__ void __launch_bounds__(kDBlock) dequant_axis0_cols_kernel(
     float sc[8], nz[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      sc[i] = meta_value(a.scale, a.scale_mm, a.meta_dtype, a.meta_group_size, g0 + i);
-      nz[i] = -meta_value(a.zero, a.zero_mm, a.meta_dtype, a.meta_group_size, g0 + i);
+      sc[i] = meta_value(a, a.scale, a.scale_mm, g0 + i);
+      nz[i] = -meta_value(a, a.zero, a.zero_mm, g0 + i);
     }
 #pragma unroll 4
     for (int j = 0; j < G; ++j) {
@@ -382,6 +387,9 @@ static void fill_dbatch(const DequantJob* jobs, int n, int64_t tile_elems, DBatc
   c.scale_mm = c.zero_mm = nullptr;
   c.meta_group_size = j0.meta_group_size > 0 ? j0.meta_group_size : 1;
   c.meta_dtype = j0.meta_dtype;
+  c.log2_meta_group = -1;
+  for (int l = 0; l < 31; ++l)
+    if ((1 << l) == c.meta_group_size) c.log2_meta_group = l;
   c.rows = c.cols = c.n = 0;
   c.group_size = j0.group_size;
   c.log2_group = 0;
