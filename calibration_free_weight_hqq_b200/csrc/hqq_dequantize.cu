@@ -132,85 +132,100 @@ __device__ __forceinline__ void store1(void* out, int64_t k, float v) {
   store_meta(out, OUT_DT, k, v);
 }
 
-// Raw bits of codes k0..k0+7 (k0 a multiple of 8): one 8..64-bit load for 8/4/2/1 bits;
-// for 3 bits the (up to) two 32-bit words they occupy, with the slot of code k0 in `off`.
-template <int NB>
-__device__ __forceinline__ uint64_t codes8_raw(const uint8_t* packed, int64_t k0, int64_t n_codes,
-                                               int& off) {
-  if constexpr (NB == 3) {
-    const uint32_t* wp = reinterpret_cast<const uint32_t*>(packed);
-    const int64_t w0 = k0 / 10;
-    off = (int)(k0 - w0 * 10);
-    const int64_t last = (k0 + 7 < n_codes ? k0 + 7 : n_codes - 1) / 10;
-    const uint32_t lo = __ldg(wp + w0);
-    const uint32_t hi = last > w0 ? __ldg(wp + w0 + 1) : 0u;
-    return (uint64_t)lo | ((uint64_t)hi << 32);
-  } else {
-    off = 0;
-    const uint8_t* src = packed + k0 * NB / 8;
-    if constexpr (NB == 8) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
-      return (uint64_t)v.x | ((uint64_t)v.y << 32);
-    } else if constexpr (NB == 4) {
-      return __ldg(reinterpret_cast<const uint32_t*>(src));
-    } else if constexpr (NB == 2) {
-      return __ldg(reinterpret_cast<const unsigned short*>(src));
-    } else {
-      return __ldg(src);
-    }
-  }
-}
-
-template <int NB>
-__device__ __forceinline__ uint32_t code_in(uint64_t raw, int off, int i) {
-  if constexpr (NB == 3) {
-    const int slot = off + i;  // 0..16: slots 10.. live in the second word
-    const uint32_t w = slot < 10 ? (uint32_t)raw : (uint32_t)(raw >> 32);
-    return (w >> (3 * (slot < 10 ? slot : slot - 10))) & 7u;
-  } else {
-    return (uint32_t)(raw >> (i * NB)) & ((1u << NB) - 1u);
-  }
-}
-
 // axis=1: 8 consecutive elements share one group and have consecutive codes. A warp covers
 // 256 consecutive elements per chunk (lane l: elements 8l .. 8l+7: their codes in one load of
 // 1..8 bytes, or two 32-bit words for 3 bits, their group's meta, one 16- or 32-byte store),
 // kD1Unroll chunks per warp per tile with every load of the tile issued before any conversion.
-// Any nbits, plain or second-level meta, any output type.
+// Any nbits, plain or second-level meta, any output type. A tile (kDTile1 elements, a multiple
+// of every group size) starts on a group and on a byte of the code stream, so its 64-bit
+// bases are formed once and the per-chunk index work is 32-bit.
 constexpr int kD1Unroll = 4;
-constexpr int64_t kDTile1 = (int64_t)kDBlock * 8 * kD1Unroll;
+constexpr int kDTile1 = kDBlock * 8 * kD1Unroll;
+
+// The 8 codes of a lane as one bit field, code j in bits NB*j .. NB*j+NB-1. `tile_codes`
+// points at the tile's first code byte (for 3 bits: `words` at the 32-bit word holding the
+// tile's first code, whose slot is r0); li is the lane's first element within the tile.
+template <int NB>
+__device__ __forceinline__ uint64_t codes8_field(const uint8_t* tile_codes, const uint32_t* words,
+                                                 int r0, int li) {
+  if constexpr (NB == 3) {
+    // 10 codes per 32-bit word (bits 30..31 unused): join the two words the 8 codes can
+    // span into 60 contiguous bits, then drop the slots before the lane's first code.
+    const uint32_t k = (uint32_t)(r0 + li);
+    const uint32_t w = k / 10u, off = k - 10u * w;
+    const uint32_t lo = __ldg(words + w);
+    const uint32_t hi = off >= 3u ? __ldg(words + w + 1) : 0u;  // code 8 is in the next word
+    return (((uint64_t)hi << 30) | (lo & 0x3FFFFFFFu)) >> (3u * off);
+  } else if constexpr (NB == 8) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(tile_codes + li));
+    return (uint64_t)v.x | ((uint64_t)v.y << 32);
+  } else if constexpr (NB == 4) {
+    return __ldg(reinterpret_cast<const uint32_t*>(tile_codes + li / 2));
+  } else if constexpr (NB == 2) {
+    return __ldg(reinterpret_cast<const unsigned short*>(tile_codes + li / 4));
+  } else {
+    return __ldg(tile_codes + li / 8);
+  }
+}
+
+// Code j of a field as the fp32 bit pattern 2^23 + code (the exact value 2^23 + code).
+template <int NB>
+__device__ __forceinline__ float code_magic(uint64_t field, int j) {
+  if constexpr (NB == 8) {
+    const uint32_t w = j < 4 ? (uint32_t)field : (uint32_t)(field >> 32);
+    return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540 + (j & 3)));
+  } else {
+    return __uint_as_float(((uint32_t)(field >> (NB * j)) & ((1u << NB) - 1u)) | 0x4B000000u);
+  }
+}
 
 template <int NB, int OUT_DT, int MAXB>
 __global__ void __launch_bounds__(kDBlock) dequant_axis1_kernel(
     const __grid_constant__ DBatch<MAXB> batch) {
   const int64_t total = batch.tile_start[batch.n];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float2 neg_magic = make_float2(-8388608.0f, -8388608.0f);
   for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
     int64_t local;
     const DArgs a = batch_args(batch, t, &local);
-    const int64_t base = local * kDTile1 + (int64_t)warp * (kD1Unroll * 256) + lane * 8;
-    uint64_t raw[kD1Unroll];
-    int off[kD1Unroll];
+    const int64_t e0 = local * kDTile1;  // the tile's first element
+    const int64_t left = a.n - e0;
+    const int rem = left < kDTile1 ? (int)left : kDTile1;
+    const uint8_t* tile_codes = a.packed + (NB == 3 ? 0 : e0 / 8 * NB);
+    const int64_t w0 = NB == 3 ? e0 / 10 : 0;
+    const int r0 = NB == 3 ? (int)(e0 - 10 * w0) : 0;
+    const uint32_t* words = reinterpret_cast<const uint32_t*>(a.packed) + w0;
+    const int64_t g0 = e0 >> a.log2_group;
+    const int lane0 = warp * (kD1Unroll * 256) + lane * 8;
+    uint64_t field[kD1Unroll];
     float sc[kD1Unroll], zr[kD1Unroll];
 #pragma unroll
     for (int u = 0; u < kD1Unroll; ++u) {
-      const int64_t i = base + u * 256;
-      if (i < a.n) {  // n and G are multiples of 8: a lane's 8 elements share one group
-        raw[u] = codes8_raw<NB>(a.packed, i, a.n, off[u]);
-        const int64_t g = i >> a.log2_group;
+      const int li = lane0 + u * 256;
+      if (li < rem) {  // n and G are multiples of 8: a lane's 8 elements share one group
+        field[u] = codes8_field<NB>(tile_codes, words, r0, li);
+        const int64_t g = g0 + (li >> a.log2_group);
         sc[u] = meta_value(a, a.scale, a.scale_mm, g);
         zr[u] = meta_value(a, a.zero, a.zero_mm, g);
       }
     }
 #pragma unroll
     for (int u = 0; u < kD1Unroll; ++u) {
-      const int64_t i = base + u * 256;
-      if (i < a.n) {
+      const int li = lane0 + u * 256;
+      if (li < rem) {
+        // (code - zero) * scale, each operation rounded once as in the scalar form: the
+        // subtraction of 2^23 is exact, x - z equals x + (-z), and the pair instructions
+        // round each lane like the scalar ones
+        const float2 nz = make_float2(-zr[u], -zr[u]), s2 = make_float2(sc[u], sc[u]);
         float v[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          v[j] = __fmul_rn(__fsub_rn(u2f_small(code_in<NB>(raw[u], off[u], j)), zr[u]), sc[u]);
-        store8<OUT_DT>(a.out, i, v);
+        for (int j = 0; j < 8; j += 2) {
+          const float2 m = make_float2(code_magic<NB>(field[u], j), code_magic<NB>(field[u], j + 1));
+          const float2 r = __fmul2_rn(__fadd2_rn(__fadd2_rn(m, neg_magic), nz), s2);
+          v[j] = r.x;
+          v[j + 1] = r.y;
+        }
+        store8<OUT_DT>(a.out, e0 + li, v);
       }
     }
   }
