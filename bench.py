@@ -339,6 +339,38 @@ def linear_source_digest() -> str:
     return h.hexdigest()
 
 
+def capture_graph(fn):
+    """fn's launches (on the current stream) captured in a CUDA graph, after one plain run."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+        side.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    return graph
+
+
+def time_graph(graph, warmup: int, steps: int, flush) -> float:
+    """Median device time (ms) of one replay, L2 flushed (flush buffer written) before each."""
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    per = []
+    for _ in range(steps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        per.append(a.elapsed_time(b))
+    return statistics.median(per)
+
+
 def run_linear(hqq, dev, args, tokens: int = 4096):
     """The consumer of the packed format (row f2): the seven linear layers of one Llama-7B
     block (q, k, v, o [4096,4096]; gate, up [11008,4096]; down [4096,11008]) quantized to
@@ -409,29 +441,28 @@ def run_linear(hqq, dev, args, tokens: int = 4096):
             profiled = {"shape_MNK": [4096, 4096, 4096],
                         "dram_bytes": t.get("dram_bytes_per_launch_4096x4096x4096"),
                         "algorithmic_bytes": 2 * 4096 * 4096 * 2 + 4096 * 4096 // 2 + 4096 * 64 * 4}
-    # decode-sized batch: the same layers at 16 tokens take the split-K kernel; weight-read
-    # bound (0.5 B of codes + 4/64 B of bf16 scale/zero per weight from HBM)
+    # decode-sized batch: the same layers at 16 tokens take the warp-MMA decode kernel;
+    # weight-read bound (0.5 B of codes + 4/64 B of bf16 scale/zero per weight from HBM). A
+    # launch takes microseconds, less than the binding's host time, so the seven launches of a
+    # step are captured in a CUDA graph and the replay is timed (L2 flushed before each).
     dec_tokens = 16
     dec = []
     for m, X, pk, sc, zr, Y, Wd in layers:
         Xd = X[:dec_tokens].contiguous()
         Yd = torch.empty(dec_tokens, m.rows, dtype=torch.bfloat16, device=dev)
-        dec.append((m, Xd, pk, sc, zr, Yd))
-    for _ in range(args.warmup):
-        for m, Xd, pk, sc, zr, Yd in dec:
-            hqq.hqq_linear(Xd, pk, sc, zr, m.rows, Y=Yd, stream=stream)
-    dec_ms = []
-    for _ in range(args.steps):
-        flush.fill_(1)
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in dec]
-        for (a, b), (m, Xd, pk, sc, zr, Yd) in zip(evs, dec):
-            a.record(stream)
-            hqq.hqq_linear(Xd, pk, sc, zr, m.rows, Y=Yd, stream=stream)
-            b.record(stream)
-        torch.cuda.synchronize()
-        dec_ms.append(sum(a.elapsed_time(b) for a, b in evs))
-    ms_dec = statistics.median(dec_ms)
+        dec.append((m, Xd, pk, sc, zr, Yd, Wd))
+
+    def dec_fused():
+        for m, Xd, pk, sc, zr, Yd, Wd in dec:
+            hqq.hqq_linear(Xd, pk, sc, zr, m.rows, Y=Yd)
+
+    def dec_cublas():
+        for m, Xd, pk, sc, zr, Yd, Wd in dec:
+            torch.matmul(Xd, Wd.t(), out=Yd)
+
+    ms_dec = time_graph(capture_graph(dec_fused), args.warmup, args.steps, flush)
+    ms_dec_cublas = time_graph(capture_graph(dec_cublas), args.warmup, args.steps, flush)
+    dec_fused()  # leave the fused result in Yd
     wbytes = sum(m.rows * m.cols * (0.5 + 4 / 64) for m, *_ in dec)
     hbm = peaks()["hbm_gbs"]
     dec_gbs = wbytes / (ms_dec * 1e-3) / 1e9
@@ -450,15 +481,18 @@ def run_linear(hqq, dev, args, tokens: int = 4096):
                      "peak_source": f"bf16 dense, {source} (burst: the kernel is timed alone)"},
         "l2": "flushed before every step",
         "decode_16_tokens": {
-            "kernel": "w4a16_skinny_kernel (split-K over a 4-CTA cluster)",
+            "kernel": "w4a16_gemv_kernel (warp-level MMA on registers, split-K over a cluster "
+                      "of up to 8 CTAs)",
+            "timing": "CUDA graph of the 7 launches, L2 flushed before each replay",
             "ms_per_step": round(ms_dec, 4), "launches_per_step": len(dec),
+            "cublas_bf16_weight_ms_per_step": round(ms_dec_cublas, 4),
             "tflops": round(sum(2.0 * dec_tokens * m.rows * m.cols for m, *_ in dec)
                             / (ms_dec * 1e-3) / 1e12, 2),
             "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm,
                          "unit": "GB/s", "frac": round(dec_gbs / hbm, 4),
                          "algorithmic": "0.5625 B of packed codes + scale/zero per weight"}},
         "wait_timeouts": hqq.hqq_wait_timeouts(),
-        "gpu_launches": 2 * len(layers) * args.steps,
+        "gpu_launches": 3 * len(layers) * args.steps,
     }
 
 
@@ -694,7 +728,9 @@ def probe_hbm(gib: float = 1.0):
 
 def single_linear(reps: int = 10, M: int = 4096):
     """One 4096 x 4096 hqq_linear launch with M tokens (bf16, 4-bit g64): the ncu profiling
-    cases (M = 4096: the 2-SM kernel; M = 16: the split-K kernel)."""
+    cases (M = 4096: the 2-SM kernel; M = 16: the decode kernel). `reps` launches are
+    captured in one CUDA graph (a decode launch is shorter than the binding's host time) and
+    the replay is timed; the weight (8.4 MB of codes) stays in L2 between launches."""
     import calibration_free_weight_hqq_b200 as hqq
     from calibration_free_weight_hqq_b200 import synthetic
     N = K = 4096
@@ -702,13 +738,17 @@ def single_linear(reps: int = 10, M: int = 4096):
     pk, s, z = hqq.hqq_quantize(W, 4, 64, 1)
     X = synthetic.activations(M, K, seed=12, device="cuda")
     Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
-    for _ in range(2):
-        hqq.hqq_linear(X, pk, s, z, N, Y=Y)
+
+    def launches():
+        for _ in range(reps):
+            hqq.hqq_linear(X, pk, s, z, N, Y=Y)
+
+    graph = capture_graph(launches)
+    graph.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(reps):
-        hqq.hqq_linear(X, pk, s, z, N, Y=Y)
+    graph.replay()
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
@@ -717,20 +757,26 @@ def single_linear(reps: int = 10, M: int = 4096):
             "wait_timeouts": hqq.hqq_wait_timeouts()}
 
 
-def configs_table(reps: int = 3):
+def configs_table(reps: int = 5):
     """Quantize and dequantize throughput of the four smaller workloads of the pages'
     configurations (the fifth, the whole model, is the headline), one line per configuration:
     solver Gweights/s and its MUFU fraction, dequantizer algorithmic GB/s and its HBM fraction.
-    Each matrix is timed with CUDA events over `reps` launches after one warm-up."""
+    Quantize: each matrix timed with CUDA events over `reps` launches after one warm-up (a
+    launch takes milliseconds, so host gaps do not matter). Dequantize: one pass over all the
+    workload's matrices is captured in a CUDA graph (so that the microsecond launches run back
+    to back, without the binding's host time between them); L2 is flushed (256 MB write)
+    before each of `reps` timed replays, which are timed one by one and averaged."""
     import calibration_free_weight_hqq_b200 as hqq
     from calibration_free_weight_hqq_b200 import workloads
     pk = peaks()
     mufu_peak = MUFU_PER_CLK_PER_SM * N_SM * pk["sm_max_mhz"] * 1e6
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     out = []
     for wl in (workloads.single_fp16(), workloads.llama7b_block_4b(),
                workloads.llama7b_block_2b_axis0(), workloads.mlp70b_mixed()):
-        q_ms = d_ms = 0.0
+        q_ms = 0.0
         dq_bytes = 0
+        passes = []  # (q, rows, cols, params, dtype, D) per matrix
         for m in wl.matrices:
             W = workloads.make_weight(m, "cuda")
             params = hqq.make_params(m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0,
@@ -740,26 +786,46 @@ def configs_table(reps: int = 3):
             need = hqq.hqq_workspace_bytes(m.rows, m.cols, params)
             ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda") if need else None
             q = hqq.hqq_quantize_ex(W, params, workspace=ws)
-            D = torch.empty_like(W)
-
-            def timed(fn):
-                fn()
-                torch.cuda.synchronize()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                for _ in range(reps):
-                    fn()
-                e1.record()
-                torch.cuda.synchronize()
-                return e0.elapsed_time(e1) / reps
-
-            q_ms += timed(lambda: hqq.hqq_quantize_ex(W, params, out=q, workspace=ws))
-            d_ms += timed(lambda: hqq.hqq_dequantize_ex(q, m.rows, m.cols, params, out_dtype=m.dtype,
-                                                        out=D))
+            hqq.hqq_quantize_ex(W, params, out=q, workspace=ws)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                hqq.hqq_quantize_ex(W, params, out=q, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            q_ms += e0.elapsed_time(e1) / reps
+            passes.append((q, m.rows, m.cols, params, m.dtype, torch.empty_like(W)))
             ng = m.numel // m.group_size
             meta_b = 2 * ng * (1 if m.quant_meta else 2)
             dq_bytes += hqq.hqq_packed_bytes(m.rows, m.cols, m.nbits) + meta_b + 2 * m.numel
-            del W, D, q, ws
+            del W, ws
+
+        def dequantize_all():
+            for q, rows, cols, params, dt, D in passes:
+                hqq.hqq_dequantize_ex(q, rows, cols, params, out_dtype=dt, out=D)
+
+        dequantize_all()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
+                dequantize_all()
+        torch.cuda.current_stream().wait_stream(side)
+        graph.replay()
+        torch.cuda.synchronize()
+        d_ms = 0.0
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            d_ms += e0.elapsed_time(e1) / reps
+        del graph, passes
         n = wl.weights
         mufu = 2 * (wl.matrices[0].iters + 1) * n / (q_ms * 1e-3)
         gbs = dq_bytes / (d_ms * 1e-3) / 1e9
@@ -767,7 +833,8 @@ def configs_table(reps: int = 3):
                     "quantize_ms": round(q_ms, 3), "quantize_Gweights_per_s": round(n / q_ms / 1e6, 2),
                     "quantize_mufu_frac": round(mufu / mufu_peak, 4),
                     "dequantize_ms": round(d_ms, 4), "dequantize_GB_per_s": round(gbs, 1),
-                    "dequantize_hbm_frac": round(gbs / pk["hbm_gbs"], 4)})
+                    "dequantize_hbm_frac": round(gbs / pk["hbm_gbs"], 4),
+                    "dequantize_timing": "CUDA graph of one pass, L2 flushed before each replay"})
     return out
 
 

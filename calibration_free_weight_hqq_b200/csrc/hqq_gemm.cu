@@ -8,16 +8,20 @@
 // the activation dtype exactly as hqq_dequantize writes it; Y[m, n] = dtype(Σ_k X[m,k]·W'[n,k]
 // accumulated in fp32 (+ bias[n])).
 //
-// Two kernels, picked by the number of rows M of X (tokens):
+// Three kernels, picked by the number of rows M of X (tokens):
 //   * w4a16_gemm_2sm_kernel (M > 128): a CTA pair computes a 512 x 256 output tile with the
 //     2-SM tensor-core MMA; each CTA dequantizes its own 128 rows of the W' tile (description
 //     at the kernel).
-//   * w4a16_skinny_kernel (M <= 128, decode-sized batches): the roles swap - W' (128 rows per
-//     CTA) is the MMA's M operand and the tokens its N - and a cluster of 8 CTAs splits K,
-//     reducing the partial sums over distributed shared memory (description at the kernel).
-// Every wait is bounded (about two seconds of %globaltimer); on expiry the CTA raises an abort
-// flag, counts a timeout in g_gemm_timeouts, skips its remaining work, waits (bounded) for
-// its own asynchronous operations and frees its TMEM.
+//   * w4a16_skinny_kernel (16 < M <= 128): the roles swap - W' (128 rows per CTA) is the
+//     MMA's M operand and the tokens its N - and a cluster of 4 CTAs splits K, reducing the
+//     partial sums over distributed shared memory (description at the kernel).
+//   * w4a16_gemv_kernel (M <= 16, decode): W' is dequantized straight into the register
+//     fragments of the warp-level MMA; a cluster of up to 8 CTAs splits K (description at the
+//     kernel); K up to 32768, larger K goes to the split-K kernel.
+// Every wait of the first two is bounded (about two seconds of %globaltimer); on expiry the
+// CTA raises an abort flag, counts a timeout in g_gemm_timeouts, skips its remaining work,
+// waits (bounded) for its own asynchronous operations and frees its TMEM. The third has no
+// waits besides the hardware cluster barrier.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -926,6 +930,233 @@ __global__ void __launch_bounds__(skinny::kThreads, 2)
   }
 }
 
+// ================================================================ decode kernel (M <= 16)
+// For up to 16 tokens the product is bound by reading the packed weight (0.5 B per weight),
+// not by the math, and the tensor-core operand round trip through shared memory of the
+// kernels above costs more than the arithmetic. Here each warp dequantizes W' straight into
+// the B fragments of the warp-level MMA (mma.sync m16n8k16, fp32 accumulation) in registers;
+// the tokens are the MMA's M = 16 rows (zero rows past M) and X comes from shared memory.
+//   * A warp owns 16 W' rows (2 n-tiles of 8) and a K-slice; 8 warps per CTA share the slice
+//     (about 100 registers a thread: 16 warps per SM); a cluster of S CTAs (S = 1, 2, 4 or 8,
+//     along x) splits K, one slice per CTA.
+//   * k-blocks of 128: lane (g, t) (g = lane / 4, t = lane % 4) loads, per n-tile, the 16 code
+//     bytes of row 8r + g at k = 32t .. 32t+31 (one group: t / 2) and that group's (scale,
+//     zero); the loads of the next 4 k-blocks are in flight while one is converted.
+//   * The contraction order inside a k-block is permuted (the same permutation on both
+//     operands): MMA step s (0..7) takes k = 32t + 4s + {0, 1, 2, 3} at the k slots
+//     {2t, 2t+1, 2t+8, 2t+9} that lane t holds, so each lane's 8 codes of one 32-bit word give
+//     the B fragments of two steps and its X fragments are 16-byte pieces of one token row.
+//     X is staged in shared memory with those pieces reordered so that the fragment loads are
+//     free of bank conflicts (rows padded to 64 mod 128 bytes).
+//   * Partial sums go over distributed shared memory to the CTA of the cluster that owns the
+//     rows (128 / S rows each), which adds the S slots in rank order (deterministic), adds bias,
+//     rounds once and stores. No waits other than the cluster barrier.
+#ifndef HQQ_GEMV_WARPS
+#define HQQ_GEMV_WARPS 8
+#endif
+#ifndef HQQ_GEMV_NT
+#define HQQ_GEMV_NT 2
+#endif
+#ifndef HQQ_GEMV_DEPTH
+#define HQQ_GEMV_DEPTH 4
+#endif
+namespace gemv {
+constexpr int kWarps = HQQ_GEMV_WARPS;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kNT = HQQ_GEMV_NT;             // n-tiles (8 W' rows) per warp
+constexpr int kRowsCta = kWarps * kNT * 8;   // 128
+constexpr int kLgRowsCta = kRowsCta == 256 ? 8 : kRowsCta == 128 ? 7 : kRowsCta == 64 ? 6 : 5;
+static_assert((1 << kLgRowsCta) == kRowsCta, "power-of-two CTA rows");
+constexpr int kKB = 128;                     // k per k-block
+constexpr int kDepth = HQQ_GEMV_DEPTH;       // k-blocks of codes in flight per warp
+constexpr int kMaxKbPerSlice = 32;           // X tile <= 16 x 8256 B
+constexpr int kMaxM = 16;
+constexpr uint32_t kRedBytes = kRowsCta * 16 * 4;
+__host__ __device__ constexpr uint32_t x_row_bytes(int kb_per) { return kb_per * 256 + 64; }
+__host__ __device__ constexpr uint32_t smem_bytes(int kb_per) {
+  return 16 * x_row_bytes(kb_per) + kRedBytes;
+}
+}  // namespace gemv
+
+template <bool F16>
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  if constexpr (F16) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  } else {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+}
+
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// grid (S, ceil(N / 128)), cluster (S, 1, 1) with S = 2^lg_s; kb_per = k-blocks per slice;
+// M <= 16.
+template <bool F16, int MT>
+__global__ void __launch_bounds__(gemv::kThreads) w4a16_gemv_kernel(
+    const void* __restrict__ X, const uint8_t* __restrict__ packed, const GemmArgs args,
+    int lg_s, int kb_per) {
+  using namespace gemv;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int rank = static_cast<int>(cluster_rank());
+  const int M = args.M, N = args.N, K = args.K;
+  const int nkb = (K + kKB - 1) / kKB;
+  const int kb0 = rank * kb_per;
+  const int nloc = max(0, min(kb_per, nkb - kb0));  // k-blocks of this slice
+  const int row_cta = static_cast<int>(blockIdx.y) * kRowsCta;
+  const int64_t row_bytes = K / 2, groups_per_row = K / 64;
+  constexpr int kMsz = MT == kF32 ? 4 : 2;
+  const uint8_t* sc_base = static_cast<const uint8_t*>(args.scale);
+  const uint8_t* zr_base = static_cast<const uint8_t*>(args.zero);
+
+  // this lane's n-tile rows (8r + g of the warp's 16) at the slice start: code and meta
+  // pointers; invalid rows read nothing (codes and meta 0 -> W' = +0)
+  const uint8_t* crow[kNT];
+  const uint8_t* srow[kNT];
+  const uint8_t* zrow[kNT];
+  bool rin[kNT];
+#pragma unroll
+  for (int r = 0; r < kNT; ++r) {
+    const int row = row_cta + warp * (kNT * 8) + 8 * r + g;
+    rin[r] = row < N;
+    crow[r] = packed + row * row_bytes + static_cast<int64_t>(kb0) * 64 + 16 * t;
+    const int64_t gi = row * groups_per_row + 2 * static_cast<int64_t>(kb0) + (t >> 1);
+    srow[r] = sc_base + gi * kMsz;
+    zrow[r] = zr_base + gi * kMsz;
+  }
+
+  uint4 code[kDepth][kNT];
+  uint32_t msc[kDepth][kNT], mzr[kDepth][kNT];
+  auto load_kb = [&](int i, uint4 (&c)[kNT], uint32_t (&s)[kNT], uint32_t (&z)[kNT]) {
+    const bool kin = (kb0 + i) * kKB + 32 * t < K;  // K % 64 == 0: lane t's 32 k all in or out
+#pragma unroll
+    for (int r = 0; r < kNT; ++r) {
+      if (kin && rin[r]) {
+        c[r] = __ldg(reinterpret_cast<const uint4*>(crow[r] + i * 64));
+        s[r] = meta_load<MT>(srow[r] + i * (2 * kMsz));
+        z[r] = meta_load<MT>(zrow[r] + i * (2 * kMsz));
+      } else {
+        c[r] = make_uint4(0u, 0u, 0u, 0u);
+        s[r] = 0u;
+        z[r] = 0u;
+      }
+    }
+  };
+#pragma unroll
+  for (int i = 0; i < kDepth; ++i)
+    if (i < nloc) load_kb(i, code[i], msc[i], mzr[i]);
+
+  // X[0..15][slice] -> shared memory: 16-byte piece q (k = 8q within the slice) of token m at
+  // m * rs + (q / 16) * 256 + (q % 4) * 64 + ((q / 4) % 4) * 16; zeros past M and past K
+  const uint32_t rs = x_row_bytes(kb_per);
+  {
+    // asynchronous 16-byte copies (all issued before one wait; 0 source bytes = zero fill);
+    // thread = (token m = tid / kTpr, piece column tid % kTpr)
+    constexpr int kTpr = kThreads / 16;
+    const int m = threadIdx.x / kTpr;
+    const int kc0 = kb0 * kKB;
+    const bool mrow = m < M;
+    const unsigned short* xrow = static_cast<const unsigned short*>(X) +
+                                 (mrow ? static_cast<int64_t>(m) * K + kc0 : 0);
+    const uint32_t xs = smem_u32(smem) + m * rs;
+    for (int q = threadIdx.x % kTpr; q < kb_per * 16; q += kTpr) {
+      const bool in = mrow && kc0 + 8 * q < K;
+      const int kk = q & 15;
+      const uint32_t dst = xs + (q >> 4) * 256 + (kk & 3) * 64 + (kk >> 2) * 16;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
+                   "l"(xrow + (in ? 8 * q : 0)), "r"(in ? 16 : 0)
+                   : "memory");
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  }
+  __syncthreads();
+
+  float acc[kNT][4];
+#pragma unroll
+  for (int r = 0; r < kNT; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
+  const uint8_t* xa_row = smem + g * rs + t * 16;
+  const uint8_t* xb_row = smem + (g + 8) * rs + t * 16;
+
+  for (int base = 0; base < nloc; base += kDepth) {
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d) {
+      const int i = base + d;
+      if (i < nloc) {
+        float2 nz2[kNT], sc2[kNT];
+#pragma unroll
+        for (int r = 0; r < kNT; ++r) {
+          const float sc = meta_f32<MT>(msc[d][r]), z = meta_f32<MT>(mzr[d][r]);
+          nz2[r] = make_float2(-z, -z);
+          sc2[r] = make_float2(sc, sc);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          // word j: k = 32t + 8j .. +7 -> steps 2j (k +0..3) and 2j+1 (k +4..7)
+          const uint4 xa = *reinterpret_cast<const uint4*>(xa_row + i * 256 + j * 64);
+          const uint4 xb = *reinterpret_cast<const uint4*>(xb_row + i * 256 + j * 64);
+#pragma unroll
+          for (int r = 0; r < kNT; ++r) {
+            const uint32_t w = j == 0 ? code[d][r].x : j == 1 ? code[d][r].y
+                             : j == 2 ? code[d][r].z : code[d][r].w;
+            const uint4 o = dequant8<F16>(w, nz2[r], sc2[r]);
+            mma_16816<F16>(acc[r], xa.x, xb.x, xa.y, xb.y, o.x, o.y);
+            mma_16816<F16>(acc[r], xa.z, xb.z, xa.w, xb.w, o.z, o.w);
+          }
+        }
+        if (i + kDepth < nloc) load_kb(i + kDepth, code[d], msc[d], mzr[d]);
+      }
+    }
+  }
+
+  // partial sums -> the owner CTA's slot for this rank: red[(src * RPO + row_local) * 16 + m]
+  const int S = 1 << lg_s, lg_rpo = kLgRowsCta - lg_s, rpo = kRowsCta >> lg_s;
+  const uint32_t red_local = smem_u32(smem + 16 * rs);
+#pragma unroll
+  for (int r = 0; r < kNT; ++r) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int rho = warp * (kNT * 8) + 8 * r + 2 * t + (e & 1);
+      const int m = g + 8 * (e >> 1);
+      const int owner = rho >> lg_rpo, rl = rho & (rpo - 1);
+      const uint32_t off = static_cast<uint32_t>(((rank * rpo + rl) * 16 + m) * 4);
+      st_cluster_f32(cluster_addr(red_local + off, static_cast<uint32_t>(owner)), acc[r][e]);
+    }
+  }
+  cluster_sync();
+
+  // owner: rows row_cta + rank * rpo .. + rpo - 1, every token < M, two rows per store
+  typedef typename std::conditional<F16, __half, __nv_bfloat16>::type T;
+  const float* red = reinterpret_cast<const float*>(smem + 16 * rs);
+  const unsigned short* bias = reinterpret_cast<const unsigned short*>(args.bias);
+  const int nbase = row_cta + rank * rpo;
+  for (int idx = threadIdx.x; idx < (M << (lg_rpo - 1)); idx += kThreads) {
+    const int m = idx >> (lg_rpo - 1), pr = 2 * (idx & ((rpo >> 1) - 1));
+    if (nbase + pr >= N) continue;
+    float v0 = 0.0f, v1 = 0.0f;
+    for (int src = 0; src < S; ++src) {  // fixed order
+      v0 = __fadd_rn(v0, red[(src * rpo + pr) * 16 + m]);
+      v1 = __fadd_rn(v1, red[(src * rpo + pr + 1) * 16 + m]);
+    }
+    if (bias != nullptr) {
+      v0 = __fadd_rn(v0, F16 ? f16_bits_to_f32(bias[nbase + pr]) : bf16_bits_to_f32(bias[nbase + pr]));
+      v1 = __fadd_rn(v1, F16 ? f16_bits_to_f32(bias[nbase + pr + 1])
+                             : bf16_bits_to_f32(bias[nbase + pr + 1]));
+    }
+    *reinterpret_cast<uint32_t*>(reinterpret_cast<T*>(args.Y) + static_cast<int64_t>(m) * N +
+                                 nbase + pr) = pack2_16<F16 ? kF16 : kBF16>(v0, v1);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -977,6 +1208,25 @@ cudaError_t launch_typed(const GemmJob& job, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   CUtensorMap mx, mw;
+  const int nkb = static_cast<int>((job.K + gemv::kKB - 1) / gemv::kKB);
+  const int S = nkb >= 16 ? 8 : nkb >= 8 ? 4 : nkb >= 4 ? 2 : 1;
+  const int kb_per = (nkb + S - 1) / S;
+  if (job.M <= gemv::kMaxM && kb_per <= gemv::kMaxKbPerSlice &&
+      (job.N + gemv::kRowsCta - 1) / gemv::kRowsCta <= 65535) {
+    const uint32_t smem = gemv::smem_bytes(kb_per);
+    cudaError_t e = cudaFuncSetAttribute(w4a16_gemv_kernel<F16, MT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(gemv::smem_bytes(gemv::kMaxKbPerSlice)));
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(static_cast<unsigned>(S),
+                       static_cast<unsigned>((job.N + gemv::kRowsCta - 1) / gemv::kRowsCta));
+    cfg.blockDim = dim3(gemv::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    const uint8_t* packed = job.packed;
+    const int lg_s = S == 8 ? 3 : S == 4 ? 2 : S == 2 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, w4a16_gemv_kernel<F16, MT>, job.X, packed, a, lg_s, kb_per);
+  }
   if (job.M <= skinny::kMaxM) {
     const int ntok = static_cast<int>(
         (std::min<int64_t>(job.M, skinny::kTokMax) + 15) / 16 * 16);

@@ -184,7 +184,7 @@ def test_linear_meta_views_with_odd_offsets():
 
 
 def test_linear_skinny_one_hot_spans_every_k_slice():
-    # M <= 128 takes the split-K kernel (8 CTAs per W' tile, each a slice of K): one-hot rows
+    # 16 < M <= 128 takes the split-K kernel (4 CTAs per W' tile, each a slice of K): one-hot rows
     # picking k = 5m + 3 reach every slice; each output is one product with 1, so Y must be
     # the dequantized weight's columns exactly (partial sums of the other slices are +0)
     N, K, M = 264, 1024, 100
@@ -215,6 +215,56 @@ def test_linear_skinny_is_deterministic():
     codes, scale, zero, dev = make_layer(N, K, 8)
     X = make_x(M, K, 9, "f16")
     dev16 = make_layer(N, K, 8, "f16")[3]
+    a = run_linear(X, dev16, N, "f16", "f16")
+    b = run_linear(X, dev16, N, "f16", "f16")
+    assert np.array_equal(a, b)
+
+
+def test_linear_decode_one_hot_spans_every_k_slice():
+    # M <= 16 takes the warp-MMA decode kernel: K = 2112 is 16.5 k-blocks of 128, split over a
+    # cluster of 8 CTAs (3 k-blocks each, the last slices partial or empty, the last k-block
+    # half). One-hot rows picking k = 131m + 7 reach every non-empty slice and every position
+    # of the in-block permutation; each output is one product with 1: Y must be the
+    # dequantized weight's columns exactly
+    N, K, M = 264, 2112, 16
+    codes, scale, zero, dev = make_layer(N, K, 32)
+    ks = 131 * np.arange(M) + 7
+    X = torch.zeros(M, K, dtype=torch.bfloat16)
+    X[torch.arange(M), torch.from_numpy(ks)] = 1.0
+    Y = run_linear(X, dev, N, "bf16", "bf16")
+    Wd = oracle.round_to_dtype(oracle.dequantize(codes, scale, zero, N, K, 64, 1), "bf16")
+    assert np.array_equal(Y, Wd[:, ks].T.astype(np.float64))
+    # every k of one k-block through the permutation: token m picks k = 128 + m, 144 + m, ..
+    for base in (128, 2048):
+        ks = base + np.arange(16) * (4 if base == 128 else 1)
+        X = torch.zeros(M, K, dtype=torch.bfloat16)
+        X[torch.arange(M), torch.from_numpy(ks)] = 1.0
+        Y = run_linear(X, dev, N, "bf16", "bf16")
+        assert np.array_equal(Y, Wd[:, ks].T.astype(np.float64))
+
+
+@pytest.mark.parametrize("M,N,K,dtype,meta,with_bias", [
+    (1, 8, 64, "bf16", "bf16", False),        # one CTA, one half k-block
+    (5, 136, 576, "f16", "f32", True),        # 2 slices, ragged row tile, half k-block
+    (16, 264, 2112, "bf16", "f16", True),     # 8 slices, two of them empty
+    (9, 1024, 4096, "f16", "f16", False),
+    (3, 256, 32768, "bf16", "bf16", True),    # the largest K the decode kernel takes
+    (2, 128, 32832, "bf16", "bf16", False),   # one k-block more: the split-K kernel
+])
+def test_linear_decode_matches_oracle(M, N, K, dtype, meta, with_bias):
+    codes, scale, zero, dev = make_layer(N, K, 500 + M + N + K, meta)
+    X = make_x(M, K, 60 + M, dtype)
+    bias = make_x(1, N, 61, dtype)[0] if with_bias else None
+    Y = run_linear(X, dev, N, dtype, meta, bias)
+    worst, same = check_against_oracle(Y, X, codes, scale, zero, N, K, dtype, bias)
+    assert same > 0.9, same
+    assert_no_timeouts()
+
+
+def test_linear_decode_is_deterministic():
+    N, K, M = 1024, 4096, 11
+    dev16 = make_layer(N, K, 12, "f16")[3]
+    X = make_x(M, K, 13, "f16")
     a = run_linear(X, dev16, N, "f16", "f16")
     b = run_linear(X, dev16, N, "f16", "f16")
     assert np.array_equal(a, b)
