@@ -838,6 +838,50 @@ def configs_table(reps: int = 5):
     return out
 
 
+def run_mixed_model(args):
+    """Per-layer mixed precision (row f1's per-matrix configurations): the whole Llama-7B-shaped
+    model with block 0 at 8-bit g128, attention at 4-bit g64 and MLP at 2-bit g16
+    (workloads.llama7b_model_mixed). A step is hqq_quantize_mixed over all 224 matrices (one
+    batched solver launch per configuration) and hqq_dequantize_mixed back to bf16; CUDA events
+    around each step on the launching stream; inputs 13 GB, above L2."""
+    import calibration_free_weight_hqq_b200 as hqq
+    from calibration_free_weight_hqq_b200 import workloads
+    wl = workloads.llama7b_model_mixed()
+    Ws = [workloads.make_weight(m, "cuda") for m in wl.matrices]
+    cfgs = [hqq.make_params(m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0, m.kappa,
+                            w_dtype=m.dtype) for m in wl.matrices]
+    outs = hqq.hqq_quantize_mixed(Ws, cfgs)
+    shapes = [tuple(W.shape) for W in Ws]
+    D = hqq.hqq_dequantize_mixed(outs, shapes, cfgs)
+
+    bq, bd = hqq.matrix_batch(Ws, outs), hqq.matrix_batch(D, outs)
+
+    def step():
+        hqq.hqq_quantize_mixed(Ws, cfgs, outs=outs, batch=bq)
+        hqq.hqq_dequantize_mixed(outs, shapes, cfgs, W_out=D, batch=bd)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    per = []
+    for _ in range(args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        step()
+        b.record()
+        torch.cuda.synchronize()
+        per.append(a.elapsed_time(b))
+    ms = statistics.median(per)
+    groups = hqq.hqq_mixed_plan(cfgs)[1]
+    counts = {}
+    for m in wl.matrices:
+        counts[f"{m.nbits}b_g{m.group_size}"] = counts.get(f"{m.nbits}b_g{m.group_size}", 0) + 1
+    return {"metric": "HQQ quantize+dequantize Gweights/s, mixed per-layer configurations",
+            "value": round(wl.weights / ms / 1e6, 3), "unit": "Gweights/s",
+            "workload": wl.name, "weights": wl.weights, "matrices_per_config": counts,
+            "ms_per_step": round(ms, 3), "launches_per_step": 2 * groups, "steps": args.steps}
+
+
 def single(kind: str, reps: int = 10):
     """One [16384, 8192] bf16 matrix (134M weights, 268 MB: larger than L2), 4-bit g64:
     time `reps` solver or dequantize launches after warm-up (the small case the ncu
@@ -889,6 +933,8 @@ def main():
                     help="measure HBM read-only, write-only and copy bandwidth and exit")
     ap.add_argument("--configs", action="store_true",
                     help="quantize/dequantize throughput of the four smaller configurations")
+    ap.add_argument("--mixed", action="store_true",
+                    help="whole model with per-layer configurations (8/4/2 bits) and exit")
     ap.add_argument("--single", choices=["quantize", "dequantize", "linear", "decode"],
                     help="time one [16384,8192] matrix, one 4096^3 linear layer, or one "
                          "4096x4096 layer at 16 tokens (the profiling cases), and exit")
@@ -902,6 +948,9 @@ def main():
     if args.configs:
         for line in configs_table():
             print(json.dumps(line), flush=True)
+        return
+    if args.mixed:
+        print(json.dumps(run_mixed_model(args)), flush=True)
         return
     if args.single:
         if args.single in ("linear", "decode"):

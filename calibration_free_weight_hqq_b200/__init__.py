@@ -97,6 +97,12 @@ def lib() -> ctypes.CDLL:
                                                ctypes.POINTER(HQQParams), P]
             L.hqq_dequantize_batched.argtypes = [ctypes.POINTER(HQQMatrix), i32,
                                                  ctypes.POINTER(HQQParams), i32, P]
+            L.hqq_quantize_mixed.argtypes = [ctypes.POINTER(HQQMatrix),
+                                             ctypes.POINTER(HQQParams), i32, P]
+            L.hqq_dequantize_mixed.argtypes = [ctypes.POINTER(HQQMatrix),
+                                               ctypes.POINTER(HQQParams), i32, i32, P]
+            L.hqq_mixed_plan.argtypes = [ctypes.POINTER(HQQParams), i32,
+                                         ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
             L.hqq_quantize_meta.argtypes = [P, i32, i64, i32, P, P, P]
             L.hqq_dequantize_meta.argtypes = [P, P, i64, i32, P, P]
             L.hqq_linear.argtypes = [P, i64, i64, i32, P, P, P, P, i64,
@@ -107,7 +113,8 @@ def lib() -> ctypes.CDLL:
             for f in ("hqq_quantize", "hqq_dequantize", "hqq_quantize_ex", "hqq_dequantize_ex",
                       "hqq_quantize_meta", "hqq_dequantize_meta", "hqq_quantize_ex_noalloc",
                       "hqq_quantize_batched", "hqq_dequantize_batched", "hqq_linear",
-                      "hqq_wait_timeouts", "hqq_mxfp4_quantize", "hqq_mxfp4_dequantize"):
+                      "hqq_wait_timeouts", "hqq_mxfp4_quantize", "hqq_mxfp4_dequantize",
+                      "hqq_quantize_mixed", "hqq_dequantize_mixed", "hqq_mixed_plan"):
                 getattr(L, f).restype = i32
             L.hqq_packed_bytes.argtypes = [i64, i64, i32, i32, i32]
             L.hqq_packed_bytes.restype = sz
@@ -321,6 +328,52 @@ def hqq_dequantize_batched(outs, shapes, params: HQQParams, out_dtype=torch.bflo
                                       _TORCH_DT.get(W_out[0].dtype if W_out else out_dtype, -1),
                                       _stream(stream))
     _check(st, "hqq_dequantize_batched")
+    return W_out
+
+
+def _params_array(params_list):
+    arr = (HQQParams * len(params_list))()
+    for i, p in enumerate(params_list):
+        arr[i] = p
+    return arr
+
+
+def hqq_mixed_plan(params_list):
+    """The grouping of a mixed call (host only): (group index per matrix, number of groups)."""
+    n = len(params_list)
+    g = (ctypes.c_int * max(n, 1))()
+    k = ctypes.c_int(0)
+    _check(lib().hqq_mixed_plan(_params_array(params_list), n, g, ctypes.byref(k)),
+           "hqq_mixed_plan")
+    return [g[i] for i in range(n)], k.value
+
+
+def hqq_quantize_mixed(Ws, params_list, *, outs=None, batch=None, stream=None):
+    """Quantize a list of 2-D CUDA weights, weight i with its own configuration params_list[i]
+    (per-layer mixed precision), one batched launch per distinct configuration. Returns the
+    list of (packed, scale, zero). `batch` = matrix_batch(Ws, outs), built once, skips the
+    per-call marshalling."""
+    if outs is None:
+        outs = [alloc_outputs([tuple(W.shape)], p, W.device)[0] for W, p in zip(Ws, params_list)]
+    if batch is None:
+        batch = matrix_batch(Ws, outs)
+    st = lib().hqq_quantize_mixed(batch, _params_array(params_list), len(Ws), _stream(stream))
+    _check(st, "hqq_quantize_mixed")
+    return outs
+
+
+def hqq_dequantize_mixed(outs, shapes, params_list, out_dtype=torch.bfloat16, *, W_out=None,
+                         batch=None, stream=None):
+    """Dequantize (packed, scale, zero) i with params_list[i] into new (or given) [rows, cols]
+    tensors of out_dtype (`batch` as in hqq_quantize_mixed, over W_out and outs)."""
+    if W_out is None:
+        W_out = [torch.empty(sh, dtype=out_dtype, device=outs[0][0].device) for sh in shapes]
+    if batch is None:
+        batch = matrix_batch(W_out, outs)
+    st = lib().hqq_dequantize_mixed(batch, _params_array(params_list),
+                                    len(W_out), _TORCH_DT.get(W_out[0].dtype if W_out else out_dtype, -1),
+                                    _stream(stream))
+    _check(st, "hqq_dequantize_mixed")
     return W_out
 
 

@@ -362,6 +362,92 @@ HQQ_EXPORT hqq_status hqq_dequantize_batched(const hqq_matrix* mats, int n, cons
   return cuda_status(hqqk::launch_dequantize_batched(jobs.data(), (int)jobs.size(), stream));
 }
 
+// ---------------------------------------------------------------- mixed configurations
+// Two configurations are the same when every field that reaches a kernel is equal.
+static bool same_config(const hqq_params& a, const hqq_params& b) {
+  return a.nbits == b.nbits && a.group_size == b.group_size && a.axis == b.axis &&
+         a.iters == b.iters && a.p == b.p && a.beta0 == b.beta0 && a.kappa == b.kappa &&
+         a.w_dtype == b.w_dtype && a.meta_dtype == b.meta_dtype &&
+         a.quant_scale == b.quant_scale && a.quant_zero == b.quant_zero &&
+         a.meta_group_size == b.meta_group_size && a.flags == b.flags;
+}
+
+// group_of[i] = index (by first appearance) of the configuration of matrix i; rep[g] = the
+// first matrix of group g.
+static void plan_mixed(const hqq_params* prm, int n, std::vector<int>* group_of,
+                       std::vector<int>* rep) {
+  group_of->assign((size_t)n, -1);
+  rep->clear();
+  for (int i = 0; i < n; ++i) {
+    int g = -1;
+    for (size_t k = 0; k < rep->size(); ++k)
+      if (same_config(prm[(*rep)[k]], prm[i])) { g = (int)k; break; }
+    if (g < 0) {
+      g = (int)rep->size();
+      rep->push_back(i);
+    }
+    (*group_of)[i] = g;
+  }
+}
+
+HQQ_EXPORT hqq_status hqq_mixed_plan(const hqq_params* params, int n, int* group_of,
+                                     int* n_groups) {
+  if (n < 0 || !n_groups || (n > 0 && (!params || !group_of))) return HQQ_ERR_INVALID_ARG;
+  std::vector<int> g, rep;
+  plan_mixed(params, n, &g, &rep);
+  for (int i = 0; i < n; ++i) group_of[i] = g[(size_t)i];
+  *n_groups = (int)rep.size();
+  return HQQ_OK;
+}
+
+// Validate every matrix against its own configuration, then issue one batched call per
+// configuration group (matrices in their original order within a group).
+template <typename Batched>
+static hqq_status run_mixed(const hqq_matrix* mats, const hqq_params* prm, int n, int out_dtype,
+                            Batched batched) {
+  if (n < 0 || (n > 0 && (!mats || !prm))) return HQQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    hqq_status st = check_batch_params(&mats[i], 1, &prm[i]);
+    if (st != HQQ_OK) return st;
+    if (out_dtype < 0) {
+      if ((st = check_solver(prm[i].iters, prm[i].p, prm[i].beta0, prm[i].kappa)) != HQQ_OK)
+        return st;
+      if (!flags_ok(prm[i].flags)) return HQQ_ERR_INVALID_ARG;
+    } else if (!wdtype_ok(out_dtype)) {
+      return HQQ_ERR_UNSUPPORTED;
+    }
+    if ((st = check_matrix(mats[i], prm[i], 16, out_dtype)) != HQQ_OK) return st;
+  }
+  std::vector<int> group_of, rep;
+  plan_mixed(prm, n, &group_of, &rep);
+  std::vector<hqq_matrix> sub;
+  sub.reserve((size_t)n);
+  for (size_t g = 0; g < rep.size(); ++g) {
+    sub.clear();
+    for (int i = 0; i < n; ++i)
+      if (group_of[(size_t)i] == (int)g) sub.push_back(mats[i]);
+    const hqq_status st = batched(sub.data(), (int)sub.size(), &prm[rep[g]]);
+    if (st != HQQ_OK) return st;
+  }
+  return HQQ_OK;
+}
+
+HQQ_EXPORT hqq_status hqq_quantize_mixed(const hqq_matrix* mats, const hqq_params* params, int n,
+                                         cudaStream_t stream) {
+  return run_mixed(mats, params, n, -1, [&](const hqq_matrix* m, int k, const hqq_params* p) {
+    return hqq_quantize_batched(m, k, p, stream);
+  });
+}
+
+HQQ_EXPORT hqq_status hqq_dequantize_mixed(const hqq_matrix* mats, const hqq_params* params,
+                                           int n, hqq_dtype out_dtype, cudaStream_t stream) {
+  if (!wdtype_ok(out_dtype)) return HQQ_ERR_UNSUPPORTED;
+  return run_mixed(mats, params, n, static_cast<int>(out_dtype),
+                   [&](const hqq_matrix* m, int k, const hqq_params* p) {
+                     return hqq_dequantize_batched(m, k, p, out_dtype, stream);
+                   });
+}
+
 HQQ_EXPORT hqq_status hqq_quantize_meta(const void* meta, hqq_dtype dtype, int64_t n, int group,
                                         void* q_u8, void* mm, cudaStream_t stream) {
   if (n < 0) return HQQ_ERR_INVALID_ARG;

@@ -108,6 +108,26 @@ def llama7b_model_4b() -> Workload:
                     "group 64, axis 1, per-matrix sigma", mats)
 
 
+def llama7b_model_mixed() -> Workload:
+    """The whole Llama-7B-shaped model with per-layer configurations after the pages' recipes:
+    block 0 at 8 bits, group 128 ("HQQ tutorial" §4.2, layer_configs: the first block and the
+    output head at 8 bits, the rest at 4 bits, group 64); in blocks 1-31 the attention
+    projections at 4 bits, group 64, and the MLP at 2 bits, group 16 ("hqq-quantization skill
+    summary", dynamic_config: attention 4-bit, MLP 2-bit; "HQQ量化 skill page": 2 bits want
+    group 16). Same shapes and seeds as the uniform 4-bit model."""
+    s = _base_seed(5)
+    mats = []
+    for layer in range(32):
+        for i, (n, r, c) in enumerate(BLOCK_SHAPES):
+            idx = layer * len(BLOCK_SHAPES) + i
+            nbits, G = (8, 128) if layer == 0 else (4, 64) if i < 4 else (2, 16)
+            mats.append(Matrix(f"layers.{layer}.{n}", r, c, s + idx, torch.bfloat16, nbits, G, 1,
+                               per_layer_sigma=True))
+    return Workload("llama7b_model_bf16_mixed_8b_4b_2b",
+                    "whole Llama-7B-shaped model, bf16, axis 1: block 0 8-bit g128, attention "
+                    "4-bit g64, MLP 2-bit g16 (blocks 1-31)", mats)
+
+
 ALL = {1: single_fp16, 2: llama7b_block_4b, 3: llama7b_block_2b_axis0, 4: mlp70b_mixed,
        5: llama7b_model_4b}
 

@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define HQQ_ABI_VERSION 4
+#define HQQ_ABI_VERSION 5
 
 typedef enum {
   HQQ_OK = 0,
@@ -242,6 +242,33 @@ hqq_status hqq_quantize_batched(const hqq_matrix* mats, int n, const hqq_params*
  * hqq_quantize_batched; results identical to hqq_dequantize_ex per matrix. */
 hqq_status hqq_dequantize_batched(const hqq_matrix* mats, int n, const hqq_params* params,
                                   hqq_dtype out_dtype, cudaStream_t stream);
+
+/* Per-layer mixed precision in one call: matrix i is quantized with its own configuration
+ * params[i] (host array of n). The pages configure layers by name pattern - 8-bit group 128 for
+ * the first block and the output head, 4-bit group 64 elsewhere ("HQQ tutorial"
+ * (devpress.csdn.net) §4.2, layer_configs) - or by layer type, e.g. 4-bit attention and 2-bit
+ * MLP weights ("hqq-quantization skill summary" (nav.superapi.store), dynamic_config).
+ * Matrices whose configurations are equal in every field form one group; the groups are
+ * issued in order of first appearance, each as hqq_quantize_batched (same rules:
+ * quant_scale/quant_zero must be 0, up to 256 matrices per launch), so a model with k
+ * distinct configurations takes k batched launches (more only past 256 matrices a group).
+ * Each matrix's results are identical to hqq_quantize_ex with its configuration. Every matrix
+ * and configuration is validated before anything is launched; on an invalid argument nothing
+ * is launched. */
+hqq_status hqq_quantize_mixed(const hqq_matrix* mats, const hqq_params* params, int n,
+                              cudaStream_t stream);
+
+/* Inverse of hqq_quantize_mixed: matrix i dequantized with params[i] into its W field
+ * (out_dtype), grouped and launched like hqq_quantize_mixed; results identical to
+ * hqq_dequantize_ex per matrix. */
+hqq_status hqq_dequantize_mixed(const hqq_matrix* mats, const hqq_params* params, int n,
+                                hqq_dtype out_dtype, cudaStream_t stream);
+
+/* Host only (no device work): the grouping hqq_quantize_mixed / hqq_dequantize_mixed use.
+ * group_of (host array of n ints) receives, for each matrix, the index of its configuration
+ * group, numbered by first appearance; *n_groups their count. HQQ_ERR_INVALID_ARG on n < 0 or
+ * a null pointer that n requires. */
+hqq_status hqq_mixed_plan(const hqq_params* params, int n, int* group_of, int* n_groups);
 
 /* Second level on its own: 8-bit min/max round-to-nearest of n fp32/f16/bf16 values `meta`
  * (device) in runs of `group` values ("HQQ tutorial" (devpress.csdn.net) §3.3). Per run:

@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(L):
     assert "hqq_quantize" in names and "hqq_dequantize" in names and len(names) >= 12
     for n in names:
         assert hasattr(L, n), n
-    assert L.hqq_abi_version() == 4
+    assert L.hqq_abi_version() == 5
 
 
 def test_size_helpers_match_layout(L):
@@ -146,6 +146,50 @@ def test_batched_calls_validate_before_launch(L):
     assert L.hqq_quantize_batched(arr, 0, ctypes.byref(p), None) == OK
     odd = (hqq.HQQMatrix * 1)(hqq.HQQMatrix(FAKE + 8, 64, 128, FAKE, FAKE, FAKE))
     assert L.hqq_quantize_batched(odd, 1, ctypes.byref(p), None) == ALIGN
+
+
+def test_mixed_plan_groups_equal_configurations():
+    # the pages' per-layer recipes: 8-bit g128 for the first block / output head, 4-bit g64
+    # elsewhere ("HQQ tutorial" §4.2), 2-bit g16 MLP ("hqq-quantization skill summary")
+    c8 = hqq.make_params(8, 128)
+    c4 = hqq.make_params(4, 64)
+    c2 = hqq.make_params(2, 16)
+    c4b = hqq.make_params(4, 64)  # equal to c4 field by field: the same group
+    assert hqq.hqq_mixed_plan([c8, c4, c2, c4b, c2, c8]) == ([0, 1, 2, 1, 2, 0], 3)
+    # any field that reaches a kernel separates configurations
+    variants = [hqq.make_params(4, 64, axis=0), hqq.make_params(4, 64, iters=5),
+                hqq.make_params(4, 64, p=0.5), hqq.make_params(4, 64, w_dtype=torch.float16),
+                hqq.make_params(4, 64, meta_dtype=torch.float32),
+                hqq.make_params(4, 64, stop_at_fixed_point=True)]
+    groups, k = hqq.hqq_mixed_plan([c4] + variants)
+    assert groups == list(range(1 + len(variants))) and k == 1 + len(variants)
+    assert hqq.hqq_mixed_plan([]) == ([], 0)
+
+
+def test_mixed_calls_validate_every_matrix_before_launch(L):
+    good = hqq.HQQMatrix(FAKE, 64, 128, FAKE, FAKE, FAKE)
+    arr = (hqq.HQQMatrix * 2)(good, good)
+    ok4, bad5 = hqq.make_params(4, 64), hqq.make_params(4, 64)
+    bad5.nbits = 5
+    prm = (hqq.HQQParams * 2)(ok4, bad5)
+    assert L.hqq_quantize_mixed(arr, prm, 2, None) == UNSUPPORTED
+    assert L.hqq_dequantize_mixed(arr, prm, 2, 1, None) == UNSUPPORTED
+    # the second matrix does not fit its own configuration (cols % 256)
+    prm = (hqq.HQQParams * 2)(ok4, hqq.make_params(8, 256))
+    assert L.hqq_quantize_mixed(arr, prm, 2, None) == SHAPE
+    assert L.hqq_dequantize_mixed(arr, prm, 2, 1, None) == SHAPE
+    q = hqq.make_params(4, 64, quant_scale=True)
+    prm = (hqq.HQQParams * 2)(ok4, q)
+    assert L.hqq_quantize_mixed(arr, prm, 2, None) == UNSUPPORTED
+    prm = (hqq.HQQParams * 2)(ok4, ok4)
+    assert L.hqq_dequantize_mixed(arr, prm, 2, 7, None) == UNSUPPORTED
+    assert L.hqq_quantize_mixed(None, prm, 2, None) == INVALID
+    assert L.hqq_quantize_mixed(arr, None, 2, None) == INVALID
+    assert L.hqq_quantize_mixed(arr, prm, -1, None) == INVALID
+    assert L.hqq_quantize_mixed(arr, prm, 0, None) == OK
+    empty = (hqq.HQQMatrix * 1)(hqq.HQQMatrix(None, 0, 128, None, None, None))
+    assert L.hqq_quantize_mixed(empty, prm, 1, None) == OK
+    assert L.hqq_mixed_plan(prm, -1, None, None) == INVALID
 
 
 def test_unknown_flags_are_rejected(L):
