@@ -937,7 +937,7 @@ __global__ void __launch_bounds__(skinny::kThreads, 2)
 // the B fragments of the warp-level MMA (mma.sync m16n8k16, fp32 accumulation) in registers;
 // the tokens are the MMA's M = 16 rows (zero rows past M) and X comes from shared memory.
 //   * A warp owns 16 W' rows (2 n-tiles of 8) and a K-slice; 8 warps per CTA share the slice
-//     (about 100 registers a thread: 16 warps per SM); a cluster of S CTAs (S = 1, 2, 4 or 8,
+//     (115 registers a thread: 2 CTAs, 16 warps per SM); a cluster of S CTAs (S = 1, 2, 4 or 8,
 //     along x) splits K, one slice per CTA.
 //   * k-blocks of 128: lane (g, t) (g = lane / 4, t = lane % 4) loads, per n-tile, the 16 code
 //     bytes of row 8r + g at k = 32t .. 32t+31 (one group: t / 2) and that group's (scale,
