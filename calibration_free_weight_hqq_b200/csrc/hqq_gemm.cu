@@ -951,6 +951,8 @@ __global__ void __launch_bounds__(skinny::kThreads, 2)
 //   * Partial sums go over distributed shared memory to the CTA of the cluster that owns the
 //     rows (128 / S rows each), which adds the S slots in rank order (deterministic), adds bias,
 //     rounds once and stores. No waits other than the cluster barrier.
+// Tile shape (compile-time): warps per CTA, n-tiles per warp, k-blocks in flight. The defaults
+// were the best or equal among 4/8/16 warps, 1/2/4 n-tiles and 2/4 k-blocks on B200.
 #ifndef HQQ_GEMV_WARPS
 #define HQQ_GEMV_WARPS 8
 #endif
