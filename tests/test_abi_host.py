@@ -245,3 +245,22 @@ def test_mxfp4_validates_before_launch(L):
     assert L.hqq_mxfp4_dequantize(FAKE, FAKE, 4, 64, BF16, FAKE + 8, None) == ALIGN
     assert L.hqq_mxfp4_dequantize(FAKE, FAKE, 4, 64, U8, FAKE, None) == UNSUPPORTED
     assert L.hqq_mxfp4_dequantize(None, None, 4, 0, BF16, None, None) == OK
+
+
+def test_mixed_model_workload_is_valid_for_its_configurations():
+    # the --mixed bench workload: block 0 at 8-bit g128, attention 4-bit g64, MLP 2-bit g16;
+    # every matrix fits its own configuration and the plan makes three launch groups
+    from calibration_free_weight_hqq_b200 import workloads
+    wl = workloads.llama7b_model_mixed()
+    uniform = workloads.llama7b_model_4b()
+    assert [(m.rows, m.cols, m.seed) for m in wl.matrices] == \
+        [(m.rows, m.cols, m.seed) for m in uniform.matrices]
+    counts = {}
+    for m in wl.matrices:
+        counts[(m.nbits, m.group_size)] = counts.get((m.nbits, m.group_size), 0) + 1
+        assert hqq.hqq_num_groups(m.rows, m.cols, m.group_size, m.axis) > 0
+    assert counts == {(8, 128): 7, (4, 64): 4 * 31, (2, 16): 3 * 31}
+    cfgs = [hqq.make_params(m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0, m.kappa,
+                            w_dtype=m.dtype) for m in wl.matrices]
+    groups, k = hqq.hqq_mixed_plan(cfgs)
+    assert k == 3 and groups[:7] == [0] * 7 and groups[7:11] == [1] * 4 and groups[11:14] == [2] * 3
