@@ -59,6 +59,8 @@ def _load():
             lib.hqq_oracle_codes_at_zero.restype = None
             lib.hqq_oracle_shrink.argtypes = [f32, f32, f32]
             lib.hqq_oracle_shrink.restype = f32
+            lib.hqq_oracle_pow_pm1.argtypes = [f32, f32]
+            lib.hqq_oracle_pow_pm1.restype = f32
             lib.hqq_oracle_packed_bytes.argtypes = [i64, i32]
             lib.hqq_oracle_packed_bytes.restype = i64
             lib.hqq_oracle_pack.argtypes = [P, i64, i32, P]
@@ -142,6 +144,11 @@ def codes_at_zero(w, nbits: int, zero: float) -> np.ndarray:
     out = np.zeros(w.size, np.uint8)
     _load().hqq_oracle_codes_at_zero(_ptr(w), w.size, nbits, float(zero), _ptr(out))
     return out
+
+
+def pow_pm1(a: float, p: float) -> np.float32:
+    """a^(p-1) (a > 0) rounded once to fp32, as the solver's shrinkage and error use it."""
+    return np.float32(_load().hqq_oracle_pow_pm1(a, p))
 
 
 def shrink(r: float, beta: float, p: float) -> np.float32:

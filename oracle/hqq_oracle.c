@@ -54,6 +54,14 @@
 
 #define ORACLE_MAX_GROUP 1024
 
+/* a^(p-1) for a > 0, rounded once to fp32 (R7): the power is evaluated in fp64 and then
+ * rounded to fp32, which gives the correctly rounded fp32 value except for inputs within a
+ * few fp64 ulps of an fp32 rounding boundary (a libm powf may be an ulp off the correctly
+ * rounded value, and differently so on each platform). */
+static float pow_pm1(float a, float p) {
+  return (float)pow((double)a, (double)(p - 1.0f));
+}
+
 /* lp generalised soft-threshold of one residual value (R7, after [guide 2.1] and
  * [tutorial 2]). t = |r|^(p-1) is passed in so that the caller can reuse it for the
  * error term; t = +inf for r == 0. */
@@ -64,10 +72,13 @@ static float shrink_lp(float r, float t, float inv_beta) {
   return copysignf(m, r);
 }
 
+/* Exposed for the pins: a^(p-1) as the solver rounds it. */
+float hqq_oracle_pow_pm1(float a, float p) { return pow_pm1(a, p); }
+
 /* Exposed for the special-case pins (p = 1 is the textbook soft-threshold). */
 float hqq_oracle_shrink(float r, float beta, float p) {
   float a = fabsf(r);
-  float t = a > 0.0f ? powf(a, p - 1.0f) : INFINITY;
+  float t = a > 0.0f ? pow_pm1(a, p) : INFINITY;
   float inv_beta = 1.0f / beta;
   return shrink_lp(r, t, inv_beta);
 }
@@ -132,7 +143,7 @@ float hqq_oracle_quantize_group(const float* w, int G, int nbits, int iters, flo
       float wr = back * step;    /* dequantized weight */
       r[j] = w[j] - wr;          /* residual */
       float a = fabsf(r[j]);
-      t[j] = a > 0.0f ? powf(a, p - 1.0f) : INFINITY;
+      t[j] = a > 0.0f ? pow_pm1(a, p) : INFINITY;
       if (a > 0.0f) e += a * t[j]; /* |r|^p (R2) */
     }
     if (z_trace) z_trace[k] = z;

@@ -174,6 +174,24 @@ def test_exact_grid_group(offset, zero):
 # ---------------------------------------------------------------- shrinkage
 
 
+def test_power_is_correctly_rounded():
+    """a^(p-1) as the solver uses it is the exact power rounded once to fp32: checked against
+    a 40-digit decimal evaluation (the fp32 value must lie within half an ulp of it)."""
+    import decimal
+    ctx = decimal.Context(prec=40)
+    rng = np.random.default_rng(17)
+    a_vals = np.concatenate([rng.random(300) * 10, 10.0 ** rng.uniform(-7, 0, 300)])
+    for p in (0.5, 0.7, 0.9, 1.0):
+        pm1 = decimal.Decimal(float(np.float32(np.float32(p) - np.float32(1))))
+        for a in a_vals.astype(np.float32):
+            if not a > 0:
+                continue
+            t = oracle.pow_pm1(float(a), p)
+            exact = ctx.power(decimal.Decimal(float(a)), pm1)
+            half_ulp = decimal.Decimal(float(np.spacing(t))) / 2
+            assert abs(decimal.Decimal(float(t)) - exact) <= half_ulp, (a, p, t)
+
+
 def test_shrink_p1_is_textbook_soft_threshold():
     rng = np.random.default_rng(40)
     for r in rng.standard_normal(200).astype(F32):
