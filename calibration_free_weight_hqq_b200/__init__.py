@@ -140,17 +140,30 @@ def _check(status: int, where: str):
         raise HQQError(status, where, detail)
 
 
-def _cuda(t: torch.Tensor, name: str) -> int:
+def _cuda(t: torch.Tensor, name: str, dev: Optional[torch.device] = None) -> int:
+    """Device pointer of a contiguous CUDA tensor; with `dev`, the tensor must live there."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if dev is not None:
+        _same_device(dev, t, name)
     return t.data_ptr()
 
 
-def _stream(stream: Optional[torch.cuda.Stream]) -> int:
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return s.cuda_stream
+def _same_device(dev: torch.device, t: torch.Tensor, name: str) -> None:
+    """Every buffer of a call lives on the device of its first input: the library launches on
+    the current device, which the wrappers set to that one."""
+    if t.device != dev:
+        raise ValueError(f"{name} is on {t.device}, but this call runs on {dev}")
+
+
+def _stream(stream: Optional[torch.cuda.Stream], dev: torch.device) -> int:
+    if stream is None:
+        return torch.cuda.current_stream(dev).cuda_stream
+    if stream.device != dev:
+        raise ValueError(f"stream belongs to {stream.device}, but this call runs on {dev}")
+    return stream.cuda_stream
 
 
 def hqq_packed_bytes(rows: int, cols: int, nbits: int, group_size: int = 64, axis: int = 1) -> int:
@@ -196,6 +209,7 @@ def hqq_quantize(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: in
         raise ValueError("W must be 2-D [out_features, in_features]")
     rows, cols = W.shape
     wp = _cuda(W, "W")
+    dev = W.device
     if Wq_packed is None:
         Wq_packed = torch.empty(hqq_packed_bytes(rows, cols, nbits, group_size, axis),
                                 dtype=torch.uint8, device=W.device)
@@ -204,9 +218,11 @@ def hqq_quantize(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: in
         scale = torch.empty(ms, dtype=W.dtype, device=W.device)
     if zero is None:
         zero = torch.empty(ms, dtype=W.dtype, device=W.device)
-    st = lib().hqq_quantize(wp, _TORCH_DT.get(W.dtype, -1), rows, cols, nbits, group_size, axis,
-                            iters, p, beta0, kappa, _cuda(Wq_packed, "Wq_packed"),
-                            _cuda(scale, "scale"), _cuda(zero, "zero"), _stream(stream))
+    with torch.cuda.device(dev):
+        st = lib().hqq_quantize(wp, _TORCH_DT.get(W.dtype, -1), rows, cols, nbits, group_size,
+                                axis, iters, p, beta0, kappa, _cuda(Wq_packed, "Wq_packed", dev),
+                                _cuda(scale, "scale", dev), _cuda(zero, "zero", dev),
+                                _stream(stream, dev))
     _check(st, "hqq_quantize")
     return Wq_packed, scale, zero
 
@@ -238,13 +254,19 @@ def hqq_quantize_ex(W: torch.Tensor, params: HQQParams, *, stream=None, workspac
     need = hqq_workspace_bytes(rows, cols, params)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    st = lib().hqq_quantize_ex(
-        wp, rows, cols, ctypes.byref(params), _cuda(out["Wq_packed"], "Wq_packed"),
-        _cuda(out["scale"], "scale"), _cuda(out["zero"], "zero"),
-        out["scale_mm"].data_ptr() if out["scale_mm"] is not None else None,
-        out["zero_mm"].data_ptr() if out["zero_mm"] is not None else None,
-        workspace.data_ptr() if workspace is not None else None,
-        workspace.numel() if workspace is not None else 0, _stream(stream))
+    for k in ("scale_mm", "zero_mm"):
+        if out[k] is not None:
+            _same_device(dev, out[k], k)
+    if workspace is not None:
+        _same_device(dev, workspace, "workspace")
+    with torch.cuda.device(dev):
+        st = lib().hqq_quantize_ex(
+            wp, rows, cols, ctypes.byref(params), _cuda(out["Wq_packed"], "Wq_packed", dev),
+            _cuda(out["scale"], "scale", dev), _cuda(out["zero"], "zero", dev),
+            out["scale_mm"].data_ptr() if out["scale_mm"] is not None else None,
+            out["zero_mm"].data_ptr() if out["zero_mm"] is not None else None,
+            workspace.data_ptr() if workspace is not None else None,
+            workspace.numel() if workspace is not None else 0, _stream(stream, dev))
     _check(st, "hqq_quantize_ex")
     return out
 
@@ -271,11 +293,14 @@ def hqq_quantize_ex_noalloc(W: torch.Tensor, params: HQQParams, *, stream=None):
         "zero_mm": torch.empty((runs, 2), dtype=torch.float32, device=dev)
         if params.quant_zero else None,
     }
-    st = lib().hqq_quantize_ex_noalloc(
-        _cuda(W, "W"), rows, cols, ctypes.byref(params), _cuda(out["Wq_packed"], "Wq_packed"),
-        _cuda(out["scale"], "scale"), _cuda(out["zero"], "zero"),
-        out["scale_mm"].data_ptr() if out["scale_mm"] is not None else None,
-        out["zero_mm"].data_ptr() if out["zero_mm"] is not None else None, _stream(stream))
+    with torch.cuda.device(dev):
+        st = lib().hqq_quantize_ex_noalloc(
+            _cuda(W, "W"), rows, cols, ctypes.byref(params),
+            _cuda(out["Wq_packed"], "Wq_packed", dev), _cuda(out["scale"], "scale", dev),
+            _cuda(out["zero"], "zero", dev),
+            out["scale_mm"].data_ptr() if out["scale_mm"] is not None else None,
+            out["zero_mm"].data_ptr() if out["zero_mm"] is not None else None,
+            _stream(stream, dev))
     _check(st, "hqq_quantize_ex_noalloc")
     return out
 
@@ -298,10 +323,18 @@ def matrix_batch(Ws, outs):
     outputs of a dequantize) and their (packed, scale, zero) outs[i]; build it once and
     reuse it across calls to skip the per-call marshalling."""
     arr = (HQQMatrix * len(Ws))()
+    dev = Ws[0].device if len(Ws) else None
     for i, (W, (pk, sc, zr)) in enumerate(zip(Ws, outs)):
-        arr[i] = HQQMatrix(_cuda(W, "W"), W.shape[0], W.shape[1], _cuda(pk, "Wq_packed"),
-                           _cuda(sc, "scale"), _cuda(zr, "zero"))
+        arr[i] = HQQMatrix(_cuda(W, "W", dev), W.shape[0], W.shape[1],
+                           _cuda(pk, "Wq_packed", dev), _cuda(sc, "scale", dev),
+                           _cuda(zr, "zero", dev))
     return arr
+
+
+def _batch_device(tensors) -> torch.device:
+    if not len(tensors):
+        return torch.device("cuda", torch.cuda.current_device())
+    return tensors[0].device
 
 
 def hqq_quantize_batched(Ws, params: HQQParams, *, outs=None, batch=None, stream=None):
@@ -311,7 +344,10 @@ def hqq_quantize_batched(Ws, params: HQQParams, *, outs=None, batch=None, stream
         outs = alloc_outputs([tuple(W.shape) for W in Ws], params, Ws[0].device)
     if batch is None:
         batch = matrix_batch(Ws, outs)
-    st = lib().hqq_quantize_batched(batch, len(Ws), ctypes.byref(params), _stream(stream))
+    dev = _batch_device(Ws)
+    with torch.cuda.device(dev):
+        st = lib().hqq_quantize_batched(batch, len(Ws), ctypes.byref(params),
+                                        _stream(stream, dev))
     _check(st, "hqq_quantize_batched")
     return outs
 
@@ -324,9 +360,11 @@ def hqq_dequantize_batched(outs, shapes, params: HQQParams, out_dtype=torch.bflo
         W_out = [torch.empty(sh, dtype=out_dtype, device=outs[0][0].device) for sh in shapes]
     if batch is None:
         batch = matrix_batch(W_out, outs)
-    st = lib().hqq_dequantize_batched(batch, len(W_out), ctypes.byref(params),
-                                      _TORCH_DT.get(W_out[0].dtype if W_out else out_dtype, -1),
-                                      _stream(stream))
+    dev = _batch_device(W_out)
+    with torch.cuda.device(dev):
+        st = lib().hqq_dequantize_batched(
+            batch, len(W_out), ctypes.byref(params),
+            _TORCH_DT.get(W_out[0].dtype if W_out else out_dtype, -1), _stream(stream, dev))
     _check(st, "hqq_dequantize_batched")
     return W_out
 
@@ -357,7 +395,10 @@ def hqq_quantize_mixed(Ws, params_list, *, outs=None, batch=None, stream=None):
         outs = [alloc_outputs([tuple(W.shape)], p, W.device)[0] for W, p in zip(Ws, params_list)]
     if batch is None:
         batch = matrix_batch(Ws, outs)
-    st = lib().hqq_quantize_mixed(batch, _params_array(params_list), len(Ws), _stream(stream))
+    dev = _batch_device(Ws)
+    with torch.cuda.device(dev):
+        st = lib().hqq_quantize_mixed(batch, _params_array(params_list), len(Ws),
+                                      _stream(stream, dev))
     _check(st, "hqq_quantize_mixed")
     return outs
 
@@ -370,9 +411,11 @@ def hqq_dequantize_mixed(outs, shapes, params_list, out_dtype=torch.bfloat16, *,
         W_out = [torch.empty(sh, dtype=out_dtype, device=outs[0][0].device) for sh in shapes]
     if batch is None:
         batch = matrix_batch(W_out, outs)
-    st = lib().hqq_dequantize_mixed(batch, _params_array(params_list),
-                                    len(W_out), _TORCH_DT.get(W_out[0].dtype if W_out else out_dtype, -1),
-                                    _stream(stream))
+    dev = _batch_device(W_out)
+    with torch.cuda.device(dev):
+        st = lib().hqq_dequantize_mixed(
+            batch, _params_array(params_list), len(W_out),
+            _TORCH_DT.get(W_out[0].dtype if W_out else out_dtype, -1), _stream(stream, dev))
     _check(st, "hqq_dequantize_mixed")
     return W_out
 
@@ -383,10 +426,12 @@ def hqq_dequantize(Wq_packed, scale, zero, rows: int, cols: int, nbits: int = 4,
     """Dequantize to a [rows, cols] CUDA tensor of out_dtype."""
     if out is None:
         out = torch.empty((rows, cols), dtype=out_dtype, device=Wq_packed.device)
-    st = lib().hqq_dequantize(_cuda(Wq_packed, "Wq_packed"), _cuda(scale, "scale"),
-                              _cuda(zero, "zero"), _TORCH_DT.get(scale.dtype, -1),
-                              _TORCH_DT.get(out.dtype, -1), rows, cols, nbits, group_size, axis,
-                              _cuda(out, "out"), _stream(stream))
+    dev = Wq_packed.device
+    with torch.cuda.device(dev):
+        st = lib().hqq_dequantize(_cuda(Wq_packed, "Wq_packed"), _cuda(scale, "scale", dev),
+                                  _cuda(zero, "zero", dev), _TORCH_DT.get(scale.dtype, -1),
+                                  _TORCH_DT.get(out.dtype, -1), rows, cols, nbits, group_size,
+                                  axis, _cuda(out, "out", dev), _stream(stream, dev))
     _check(st, "hqq_dequantize")
     return out
 
@@ -397,11 +442,17 @@ def hqq_dequantize_ex(q: dict, rows: int, cols: int, params: HQQParams, out_dtyp
     if out is None:
         out = torch.empty((rows, cols), dtype=out_dtype, device=q["Wq_packed"].device)
     smm, zmm = q.get("scale_mm"), q.get("zero_mm")
-    st = lib().hqq_dequantize_ex(
-        _cuda(q["Wq_packed"], "Wq_packed"), _cuda(q["scale"], "scale"), _cuda(q["zero"], "zero"),
-        smm.data_ptr() if smm is not None else None, zmm.data_ptr() if zmm is not None else None,
-        rows, cols, ctypes.byref(params), _TORCH_DT.get(out.dtype, -1), _cuda(out, "out"),
-        _stream(stream))
+    dev = q["Wq_packed"].device
+    for name, t in (("scale_mm", smm), ("zero_mm", zmm)):
+        if t is not None:
+            _same_device(dev, t, name)
+    with torch.cuda.device(dev):
+        st = lib().hqq_dequantize_ex(
+            _cuda(q["Wq_packed"], "Wq_packed"), _cuda(q["scale"], "scale", dev),
+            _cuda(q["zero"], "zero", dev),
+            smm.data_ptr() if smm is not None else None,
+            zmm.data_ptr() if zmm is not None else None, rows, cols, ctypes.byref(params),
+            _TORCH_DT.get(out.dtype, -1), _cuda(out, "out", dev), _stream(stream, dev))
     _check(st, "hqq_dequantize_ex")
     return out
 
@@ -412,16 +463,21 @@ def hqq_quantize_meta(meta: torch.Tensor, group: int = 128, *, stream=None):
     q = torch.empty(n, dtype=torch.uint8, device=meta.device)
     mm = torch.empty((max(hqq_num_meta_groups(n, group), 0), 2), dtype=torch.float32,
                      device=meta.device)
-    st = lib().hqq_quantize_meta(_cuda(meta, "meta"), _TORCH_DT.get(meta.dtype, -1), n, group,
-                                 _cuda(q, "q"), _cuda(mm, "mm"), _stream(stream))
+    dev = meta.device
+    with torch.cuda.device(dev):
+        st = lib().hqq_quantize_meta(_cuda(meta, "meta"), _TORCH_DT.get(meta.dtype, -1), n,
+                                     group, _cuda(q, "q", dev), _cuda(mm, "mm", dev),
+                                     _stream(stream, dev))
     _check(st, "hqq_quantize_meta")
     return q, mm
 
 
 def hqq_dequantize_meta(q: torch.Tensor, mm: torch.Tensor, group: int = 128, *, stream=None):
     out = torch.empty(q.numel(), dtype=torch.float32, device=q.device)
-    st = lib().hqq_dequantize_meta(_cuda(q, "q"), _cuda(mm, "mm"), q.numel(), group,
-                                   _cuda(out, "out"), _stream(stream))
+    dev = q.device
+    with torch.cuda.device(dev):
+        st = lib().hqq_dequantize_meta(_cuda(q, "q"), _cuda(mm, "mm", dev), q.numel(), group,
+                                       _cuda(out, "out", dev), _stream(stream, dev))
     _check(st, "hqq_dequantize_meta")
     return out
 
@@ -443,10 +499,13 @@ def hqq_linear(X: torch.Tensor, Wq_packed: torch.Tensor, scale: torch.Tensor,
     X2 = X.reshape(M, K)
     if Y is None:
         Y = torch.empty(*lead, N, dtype=X.dtype, device=X.device)
-    st = lib().hqq_linear(_cuda(X2, "X"), M, K, _TORCH_DT.get(X.dtype, -1),
-                          _cuda(Wq_packed, "Wq_packed"), _cuda(scale, "scale"),
-                          _cuda(zero, "zero"), _cuda(bias, "bias") if bias is not None else None,
-                          N, ctypes.byref(params), _cuda(Y, "Y"), _stream(stream))
+    dev = X.device
+    with torch.cuda.device(dev):
+        st = lib().hqq_linear(_cuda(X2, "X"), M, K, _TORCH_DT.get(X.dtype, -1),
+                              _cuda(Wq_packed, "Wq_packed", dev), _cuda(scale, "scale", dev),
+                              _cuda(zero, "zero", dev),
+                              _cuda(bias, "bias", dev) if bias is not None else None,
+                              N, ctypes.byref(params), _cuda(Y, "Y", dev), _stream(stream, dev))
     _check(st, "hqq_linear")
     return Y
 
@@ -469,9 +528,11 @@ def hqq_mxfp4_quantize(W: torch.Tensor, *, codes: Optional[torch.Tensor] = None,
         codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=W.device)
     if scales is None:
         scales = torch.empty(rows, cols // 32, dtype=torch.uint8, device=W.device)
-    st = lib().hqq_mxfp4_quantize(_cuda(W, "W"), _TORCH_DT.get(W.dtype, -1), rows, cols,
-                                  _cuda(codes, "codes"), _cuda(scales, "scales"),
-                                  _stream(stream))
+    dev = W.device
+    with torch.cuda.device(dev):
+        st = lib().hqq_mxfp4_quantize(_cuda(W, "W"), _TORCH_DT.get(W.dtype, -1), rows, cols,
+                                      _cuda(codes, "codes", dev), _cuda(scales, "scales", dev),
+                                      _stream(stream, dev))
     _check(st, "hqq_mxfp4_quantize")
     return codes, scales
 
@@ -482,8 +543,10 @@ def hqq_mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, rows: int, c
     """Decode MXFP4 codes and scales to a [rows, cols] CUDA tensor of out_dtype."""
     if out is None:
         out = torch.empty(rows, cols, dtype=out_dtype, device=codes.device)
-    st = lib().hqq_mxfp4_dequantize(_cuda(codes, "codes"), _cuda(scales, "scales"), rows, cols,
-                                    _TORCH_DT.get(out.dtype, -1), _cuda(out, "out"),
-                                    _stream(stream))
+    dev = codes.device
+    with torch.cuda.device(dev):
+        st = lib().hqq_mxfp4_dequantize(_cuda(codes, "codes"), _cuda(scales, "scales", dev),
+                                        rows, cols, _TORCH_DT.get(out.dtype, -1),
+                                        _cuda(out, "out", dev), _stream(stream, dev))
     _check(st, "hqq_mxfp4_dequantize")
     return out

@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "../../include/hqq/hqq.h"
+#include "hqq_abi_internal.h"
 #include "hqq_kernels.h"
 
 #define HQQ_EXPORT extern "C" __attribute__((visibility("default")))
@@ -17,15 +18,31 @@ static_assert((int)HQQ_F16 == hqqk::kF16 && (int)HQQ_BF16 == hqqk::kBF16 &&
               "dtype enumerators must match");
 
 namespace {
-
 thread_local char g_last_cuda_error[256] = "";
+}  // namespace
 
-hqq_status cuda_status(cudaError_t e) {
+hqq_status hqqabi::cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return HQQ_OK;
   snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
            cudaGetErrorString(e));
   return HQQ_ERR_CUDA;
 }
+
+hqq_status hqqabi::check_device(const void* p) {
+  cudaPointerAttributes at;
+  cudaError_t e = cudaPointerGetAttributes(&at, p);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (at.type == cudaMemoryTypeUnregistered) return HQQ_ERR_INVALID_ARG;  // pageable host
+  if (at.type != cudaMemoryTypeDevice) return HQQ_OK;  // pinned host or managed memory
+  int dev = -1;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_status(e);
+  return at.device == dev ? HQQ_OK : HQQ_ERR_INVALID_ARG;
+}
+
+using hqqabi::check_device;
+using hqqabi::cuda_status;
+
+namespace {
 
 constexpr int64_t kMaxElems = int64_t(1) << 40;
 
@@ -113,10 +130,10 @@ HQQ_EXPORT size_t hqq_workspace_bytes(int64_t rows, int64_t cols, const hqq_para
   return part * ((prm->quant_scale ? 1 : 0) + (prm->quant_zero ? 1 : 0));
 }
 
-static hqq_status quantize_impl(const void* W, int64_t rows, int64_t cols, const hqq_params& prm,
-                                void* Wq_packed, void* scale, void* zero, void* scale_mm,
-                                void* zero_mm, void* workspace, size_t workspace_bytes,
-                                cudaStream_t stream) {
+hqq_status hqqabi::validate_quantize(const void* W, int64_t rows, int64_t cols,
+                                     const hqq_params& prm, const void* Wq_packed,
+                                     const void* scale, const void* zero, const void* scale_mm,
+                                     const void* zero_mm) {
   hqq_status st = check_shape(rows, cols, prm.nbits, prm.group_size, prm.axis);
   if (st != HQQ_OK) return st;
   if ((st = check_solver(prm.iters, prm.p, prm.beta0, prm.kappa)) != HQQ_OK) return st;
@@ -132,11 +149,23 @@ static hqq_status quantize_impl(const void* W, int64_t rows, int64_t cols, const
   if (!qs && !aligned(scale, msz)) return HQQ_ERR_ALIGNMENT;
   if (!qz && !aligned(zero, msz)) return HQQ_ERR_ALIGNMENT;
   if ((qs && !aligned(scale_mm, 8)) || (qz && !aligned(zero_mm, 8))) return HQQ_ERR_ALIGNMENT;
+  return HQQ_OK;
+}
+
+static hqq_status quantize_impl(const void* W, int64_t rows, int64_t cols, const hqq_params& prm,
+                                void* Wq_packed, void* scale, void* zero, void* scale_mm,
+                                void* zero_mm, void* workspace, size_t workspace_bytes,
+                                cudaStream_t stream) {
+  hqq_status st =
+      hqqabi::validate_quantize(W, rows, cols, prm, Wq_packed, scale, zero, scale_mm, zero_mm);
+  if (st != HQQ_OK || rows * cols == 0) return st;
+  const bool qs = prm.quant_scale != 0, qz = prm.quant_zero != 0;
   const size_t need = hqq_workspace_bytes(rows, cols, &prm);
   if (need > 0) {
     if (!workspace || workspace_bytes < need) return HQQ_ERR_WORKSPACE;
     if (!aligned(workspace, 16)) return HQQ_ERR_ALIGNMENT;
   }
+  if ((st = check_device(W)) != HQQ_OK) return st;
   const int64_t ng = rows * cols / prm.group_size;
 
   const size_t part = round_up((size_t)ng * 4, 256);
@@ -228,6 +257,7 @@ static hqq_status dequantize_impl(const void* Wq_packed, const void* scale, cons
     return HQQ_ERR_ALIGNMENT;
   if ((scale_mm && !aligned(scale_mm, 8)) || (zero_mm && !aligned(zero_mm, 8)))
     return HQQ_ERR_ALIGNMENT;
+  if ((st = check_device(Wq_packed)) != HQQ_OK) return st;
   hqqk::DequantJob j;
   j.packed = reinterpret_cast<const uint8_t*>(Wq_packed);
   j.scale = scale;
@@ -326,6 +356,8 @@ HQQ_EXPORT hqq_status hqq_quantize_batched(const hqq_matrix* mats, int n, const 
     jobs.push_back(j);
   }
   if (jobs.empty()) return HQQ_OK;
+  for (const hqqk::QuantJob& j : jobs)  // every matrix's arguments are valid: now its device
+    if ((st = check_device(j.W)) != HQQ_OK) return st;
   return cuda_status(hqqk::launch_quantize_batched(jobs.data(), (int)jobs.size(), stream));
 }
 
@@ -359,6 +391,8 @@ HQQ_EXPORT hqq_status hqq_dequantize_batched(const hqq_matrix* mats, int n, cons
     jobs.push_back(j);
   }
   if (jobs.empty()) return HQQ_OK;
+  for (const hqqk::DequantJob& j : jobs)
+    if ((st = check_device(j.packed)) != HQQ_OK) return st;
   return cuda_status(hqqk::launch_dequantize_batched(jobs.data(), (int)jobs.size(), stream));
 }
 
@@ -418,6 +452,11 @@ static hqq_status run_mixed(const hqq_matrix* mats, const hqq_params* prm, int n
     }
     if ((st = check_matrix(mats[i], prm[i], 16, out_dtype)) != HQQ_OK) return st;
   }
+  for (int i = 0; i < n; ++i) {  // all arguments are valid: now the devices, before any launch
+    if (mats[i].rows * mats[i].cols == 0) continue;
+    const hqq_status st = check_device(out_dtype < 0 ? mats[i].W : mats[i].Wq_packed);
+    if (st != HQQ_OK) return st;
+  }
   std::vector<int> group_of, rep;
   plan_mixed(prm, n, &group_of, &rep);
   std::vector<hqq_matrix> sub;
@@ -457,6 +496,7 @@ HQQ_EXPORT hqq_status hqq_quantize_meta(const void* meta, hqq_dtype dtype, int64
   if (n == 0) return HQQ_OK;
   if (!meta || !q_u8 || !mm) return HQQ_ERR_INVALID_ARG;
   if (!aligned(meta, dtype_size(dtype)) || !aligned(mm, 8)) return HQQ_ERR_ALIGNMENT;
+  if ((st = check_device(meta)) != HQQ_OK) return st;
   return cuda_status(hqqk::launch_quantize_meta(meta, dtype, n, group,
                                                 reinterpret_cast<uint8_t*>(q_u8),
                                                 reinterpret_cast<float*>(mm), stream));
@@ -470,6 +510,7 @@ HQQ_EXPORT hqq_status hqq_dequantize_meta(const void* q_u8, const void* mm, int6
   if (n == 0) return HQQ_OK;
   if (!q_u8 || !mm || !out_f32) return HQQ_ERR_INVALID_ARG;
   if (!aligned(mm, 8) || !aligned(out_f32, 4)) return HQQ_ERR_ALIGNMENT;
+  if ((st = check_device(q_u8)) != HQQ_OK) return st;
   return cuda_status(hqqk::launch_dequantize_meta(reinterpret_cast<const uint8_t*>(q_u8),
                                                   reinterpret_cast<const float*>(mm), n, group,
                                                   reinterpret_cast<float*>(out_f32), stream));
@@ -499,6 +540,8 @@ HQQ_EXPORT hqq_status hqq_linear(const void* X, int64_t M, int64_t K, hqq_dtype 
                 !aligned(scale, dtype_size(prm.meta_dtype)) ||
                 !aligned(zero, dtype_size(prm.meta_dtype))))
     return HQQ_ERR_ALIGNMENT;
+  const hqq_status dst = check_device(Y);
+  if (dst != HQQ_OK) return dst;
   hqqk::GemmJob j;
   j.X = X;
   j.packed = reinterpret_cast<const uint8_t*>(Wq_packed);
@@ -535,6 +578,7 @@ HQQ_EXPORT hqq_status hqq_mxfp4_quantize(const void* W, hqq_dtype dtype, int64_t
   if (rows * cols == 0) return HQQ_OK;
   if (!W || !codes || !scales) return HQQ_ERR_INVALID_ARG;
   if (!aligned(W, 16) || !aligned(codes, 4)) return HQQ_ERR_ALIGNMENT;
+  if ((st = check_device(W)) != HQQ_OK) return st;
   return cuda_status(hqqk::launch_mxfp4_quantize(W, dtype, rows * cols,
                                                  reinterpret_cast<uint8_t*>(codes),
                                                  reinterpret_cast<uint8_t*>(scales), stream));
@@ -549,6 +593,7 @@ HQQ_EXPORT hqq_status hqq_mxfp4_dequantize(const void* codes, const void* scales
   if (rows * cols == 0) return HQQ_OK;
   if (!codes || !scales || !W_out) return HQQ_ERR_INVALID_ARG;
   if (!aligned(codes, 4) || !aligned(W_out, 16)) return HQQ_ERR_ALIGNMENT;
+  if ((st = check_device(codes)) != HQQ_OK) return st;
   return cuda_status(hqqk::launch_mxfp4_dequantize(reinterpret_cast<const uint8_t*>(codes),
                                                    reinterpret_cast<const uint8_t*>(scales),
                                                    rows * cols, out_dtype, W_out, stream));

@@ -1,10 +1,11 @@
 // hqq_noalloc.cu - hqq_quantize_ex_noalloc: the second-level (8-bit scale/zero) quantize
 // path with its scratch in a fixed array compiled into the library, for callers that cannot
-// allocate device memory themselves. It forwards to hqq_quantize_ex with that array as the
-// workspace; nothing here allocates.
+// allocate device memory themselves. It validates the call exactly as hqq_quantize_ex does,
+// then forwards to it with that array as the workspace; nothing here allocates.
 #include <mutex>
 
 #include "../../include/hqq/hqq.h"
+#include "hqq_abi_internal.h"
 
 #define HQQ_EXPORT extern "C" __attribute__((visibility("default")))
 
@@ -20,8 +21,8 @@ std::mutex g_setup_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_scratch on the current device. In host code g_scratch only names a
-// host-side stand-in, so its address must come from the runtime, once per device, with that
-// device current.
+// host-side stand-in, so its address must come from the runtime: once per device (the
+// first call on it), with that device current, and then from this table.
 cudaError_t scratch_on_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -45,15 +46,21 @@ HQQ_EXPORT hqq_status hqq_quantize_ex_noalloc(const void* W, int64_t rows, int64
                                               void* scale, void* zero, void* scale_mm,
                                               void* zero_mm, cudaStream_t stream) {
   if (!params) return HQQ_ERR_INVALID_ARG;
+  // The same checks, in the same order, as hqq_quantize_ex, so that an invalid call reports
+  // the same status through either entry point; then the size, then the device of W.
+  hqq_status st = hqqabi::validate_quantize(W, rows, cols, *params, Wq_packed, scale, zero,
+                                            scale_mm, zero_mm);
+  if (st != HQQ_OK) return st;
   const size_t need = hqq_workspace_bytes(rows, cols, params);
-  if (need == (size_t)-1 || need == 0) {
-    // invalid arguments (reported by the regular path before any launch) or no scratch needed
+  if (need == 0 || rows * cols == 0)  // no second level: no scratch at all
     return hqq_quantize_ex(W, rows, cols, params, Wq_packed, scale, zero, scale_mm, zero_mm,
                            nullptr, 0, stream);
-  }
   if (need > kScratchBytes) return HQQ_ERR_WORKSPACE;
+  if ((st = hqqabi::check_device(W)) != HQQ_OK) return st;
+  // The current device is the one W lives on (checked just above).
   void* scratch = nullptr;
-  if (scratch_on_current_device(&scratch) != cudaSuccess) return HQQ_ERR_CUDA;
+  st = hqqabi::cuda_status(scratch_on_current_device(&scratch));
+  if (st != HQQ_OK) return st;
   return hqq_quantize_ex(W, rows, cols, params, Wq_packed, scale, zero, scale_mm, zero_mm,
                          scratch, kScratchBytes, stream);
 }

@@ -22,7 +22,11 @@
  *   Ownership  The caller owns every buffer. Nothing here allocates, frees or synchronises
  *              device memory or streams; all device work is enqueued on `stream`.
  *   Pointers   Arguments documented "device" must be device (or managed) memory on the
- *              current device. Host pointers there are undefined behaviour.
+ *              current device. Before it launches, each call checks its first device
+ *              argument (W, Wq_packed, X, meta, codes or Y) with cudaPointerGetAttributes
+ *              and returns HQQ_ERR_INVALID_ARG when that buffer lives on another device or
+ *              is pageable host memory; the other buffers of a call are the caller's
+ *              responsibility (host pointers there are undefined behaviour).
  *   Errors     Argument errors are returned synchronously before any launch, and nothing
  *              is written. When there is nothing to do (rows*cols == 0, n == 0) a call with
  *              otherwise valid arguments returns HQQ_OK at once; its pointers may be NULL.
@@ -192,13 +196,19 @@ hqq_status hqq_quantize_ex(const void* W, int64_t rows, int64_t cols, const hqq_
  * forbids allocation once it has started. The second level needs fp32 scratch for the scale
  * and zero of every group; this entry point takes it from a fixed array compiled into the
  * library instead of a caller-supplied workspace, and calls no allocating routine.
- *   Arguments, outputs and results are those of hqq_quantize_ex without the workspace.
- *   The array holds HQQ_NOALLOC_SCRATCH_BYTES; a call that needs more
+ *   Arguments, outputs and results are those of hqq_quantize_ex without the workspace; the
+ *   arguments are checked first, exactly as hqq_quantize_ex checks them, so an invalid call
+ *   returns the same status through either entry point.
+ *   The array holds HQQ_NOALLOC_SCRATCH_BYTES; a valid call that needs more
  *   (hqq_workspace_bytes() > HQQ_NOALLOC_SCRATCH_BYTES) returns HQQ_ERR_WORKSPACE and
  *   launches nothing. Calls without quant_scale/quant_zero use no scratch.
  *   Every GPU that loads the array holds it (32 MiB) until the process exits.
  *   The first call on a device sets up the array's device address for that device (a host
  *   runtime query, with the device current); make that first call before any stream capture.
+ *   If that query fails the call returns HQQ_ERR_CUDA and hqq_last_cuda_error() names the
+ *   error. The address is kept for the life of the process: after cudaDeviceReset() (or
+ *   anything else that replaces the device's primary context) this entry point must not be
+ *   called again in that process.
  *   All calls on a device share the one array and it keeps the last call's contents (each
  *   call writes the parts it reads first, so nothing needs clearing). Calls that overlap on
  *   the GPU - on different streams, or from different host threads, at the same time on one

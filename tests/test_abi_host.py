@@ -264,3 +264,41 @@ def test_mixed_model_workload_is_valid_for_its_configurations():
                             w_dtype=m.dtype) for m in wl.matrices]
     groups, k = hqq.hqq_mixed_plan(cfgs)
     assert k == 3 and groups[:7] == [0] * 7 and groups[7:11] == [1] * 4 and groups[11:14] == [2] * 3
+
+
+def test_binding_rejects_buffers_from_another_device():
+    # every buffer of a call must live on the device of its first input (the wrappers make
+    # that device current for the launch); the check itself needs no GPU
+    t = torch.zeros(4)
+    hqq._same_device(torch.device("cpu"), t, "scale")
+    with pytest.raises(ValueError, match="cuda:1"):
+        hqq._same_device(torch.device("cuda", 1), t, "scale")
+
+    class FakeStream:
+        device = torch.device("cuda", 0)
+        cuda_stream = 0
+    with pytest.raises(ValueError, match="stream belongs to cuda:0"):
+        hqq._stream(FakeStream(), torch.device("cuda", 1))
+    assert hqq._stream(FakeStream(), torch.device("cuda", 0)) == 0
+
+
+def test_noalloc_checks_arguments_before_its_size(L):
+    # an oversized call (59 MB of scratch needed, the array holds 32 MiB) that is also invalid
+    # reports what hqq_quantize_ex reports for it; only a valid oversized call is refused for
+    # its size
+    rows, cols = 28672, 8192
+
+    def call(W=FAKE, **kw):
+        p = hqq.make_params(**{**dict(nbits=1, group_size=32, quant_scale=True,
+                                      quant_zero=True), **kw})
+        na = L.hqq_quantize_ex_noalloc(W, rows, cols, ctypes.byref(p), FAKE, FAKE, FAKE, FAKE,
+                                       FAKE, None)
+        ex = L.hqq_quantize_ex(W, rows, cols, ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE,
+                               FAKE, 1 << 30, None)
+        return na, ex
+
+    assert call(p=0.0) == (INVALID, INVALID)
+    assert call(nbits=5) == (UNSUPPORTED, UNSUPPORTED)
+    assert call(W=FAKE_ODD) == (ALIGN, ALIGN)
+    assert call(meta_group_size=4) == (UNSUPPORTED, UNSUPPORTED)
+    assert call()[0] == WORKSPACE
