@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kDBlock) dequant_axis1_kernel(
 #pragma unroll
         for (int j = 0; j < 8; j += 2) {
           const float2 m = make_float2(code_magic<NB>(field[u], j), code_magic<NB>(field[u], j + 1));
-          const float2 r = __fmul2_rn(__fadd2_rn(__fadd2_rn(m, neg_magic), nz), s2);
+          const float2 r = fmul2_rn(fadd2_rn(fadd2_rn(m, neg_magic), nz), s2);
           v[j] = r.x;
           v[j + 1] = r.y;
         }

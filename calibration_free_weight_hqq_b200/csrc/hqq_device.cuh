@@ -32,6 +32,32 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// fp32 pairs (sm_100 add/mul .f32x2: one instruction, two lanes, each lane rounded to
+// nearest even exactly as the scalar operation), written as PTX with the explicit .rn
+// modifier. Measured on sm_100a: the float2 intrinsics (__fmul2_rn feeding __fadd2_rn) were
+// contracted into a fused multiply-add, one rounding instead of two, and so were these PTX
+// forms inside a large unrolled loop. So an f32x2 product must never feed an f32x2 addition
+// where the definition rounds both; callers keep such products scalar (__fmul_rn, which is
+// never fused). A product feeding nothing but a multiplication or a special function is safe.
+__device__ __forceinline__ float2 fadd2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // Exact fp32 -> fp64 widening built from the bit fields on the integer pipes (no conversion
 // instruction, which would share the SFU pipe with lg2/ex2). Zero and subnormal inputs, which
 // need renormalisation, take the conversion instruction.
@@ -102,7 +128,7 @@ __device__ __forceinline__ uint32_t pack2_16(float a, float b) {
 // code becomes the float 2^23 + q by placing its byte under the exponent bits (0x4B000000);
 // subtracting 2^23 is exact; q - zero is computed as q + (-zero) (identical rounding). The
 // arithmetic runs on fp32 pairs (sm_100 FADD2/FMUL2: one instruction, two lanes, the same
-// rounding as two scalar operations).
+// rounding as two scalar operations, fadd2_rn / fmul2_rn).
 template <int OUT>
 __device__ __forceinline__ uint4 dequant8_4bit(uint32_t w, float2 neg_zero, float2 scale) {
   const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
@@ -112,7 +138,7 @@ __device__ __forceinline__ uint4 dequant8_4bit(uint32_t w, float2 neg_zero, floa
   for (int b = 0; b < 4; ++b) {
     const float2 m = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7540 + b)),
                                  __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7540 + b)));
-    const float2 v = __fmul2_rn(__fadd2_rn(__fadd2_rn(m, neg_magic), neg_zero), scale);
+    const float2 v = fmul2_rn(fadd2_rn(fadd2_rn(m, neg_magic), neg_zero), scale);
     o[b] = pack2_16<OUT>(v.x, v.y);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);

@@ -24,7 +24,8 @@
 //   * Shrinkage: We_j is nonzero only where |r_j| > beta^(-1/(2-p)). A per-group bound on
 //     max|r_j| (from the group's min/max and the zero, no per-element work) proves We == 0
 //     exactly for almost every group and iteration; otherwise a per-element path computes
-//     We exactly as the definition does (fp32, powf, fp64 sum).
+//     We exactly as the definition does (fp32; the power is the fp64 power rounded once;
+//     fp64 sum).
 //   * The zero update uses the same fp64 expression as the definition,
 //     z = fp32(((double)sumQ - (double)sum(Ws) + (double)s*sum(We)) / G), with sumQ exact in
 //     fp32, so given identical codes the zero is bit-identical whatever the summation order.

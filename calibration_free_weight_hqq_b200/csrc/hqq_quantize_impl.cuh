@@ -13,10 +13,11 @@ namespace hqqk {
 
 constexpr int kQBlock = 160;  // 5 warps; kQBlock*E codes per block is a multiple of 10
 
-// Tuning knobs (compile-time): minimum resident blocks per SM, and whether to round with
+// Tuning knobs (compile-time): minimum resident blocks per SM (0: the per-shape table
+// min_blocks below; a positive value forces it for every shape), and whether to round with
 // the hardware round instruction instead of the magic-number add.
 #ifndef HQQ_MINB
-#define HQQ_MINB 4
+#define HQQ_MINB 0
 #endif
 #ifndef HQQ_USE_FRND
 #define HQQ_USE_FRND 0
@@ -26,6 +27,33 @@ constexpr int kQBlock = 160;  // 5 warps; kQBlock*E codes per block is a multipl
 #ifndef HQQ_STORE_WS
 #define HQQ_STORE_WS 1
 #endif
+// 1: run the per-element arithmetic of an evaluation on fp32 pairs (sm_100 FADD2/FMUL2: one
+// issue slot for two elements, each lane rounded exactly as the scalar operation); 0: scalar.
+#ifndef HQQ_PAIRED
+#define HQQ_PAIRED 1
+#endif
+// 1: take the zero update's exact fp32 form when it applies (no shrinkage, |S_ws| not tiny);
+// 0: always the fp64 form.
+#ifndef HQQ_F32_UPDATE
+#define HQQ_F32_UPDATE 1
+#endif
+// axis-0 group loader: 2 = per-warp shared-memory tiles filled with 16-byte loads (no block
+// barrier), 1 = one tile per block (block barrier), 0 = each lane loads its column directly
+// (2- or 4-byte loads, one per element). The tiles apply where the shape allows them.
+#ifndef HQQ_AXIS0_TILE
+#define HQQ_AXIS0_TILE 2
+#endif
+
+// Resident blocks per SM the register budget is sized for (measured on B200, every shape of
+// the shipped workloads): with 32 elements per lane the raw and scaled weights take 48
+// registers, and 3 blocks (128 registers a thread, no spills) ran faster than 4 (96, spills)
+// for groups of 64 and more; groups of 32 (one lane each) ran fastest with 5 blocks, whose
+// extra warps hide the lanes that take the exact shrinkage path; with 16 or fewer elements
+// per lane 4 blocks fit without spills.
+template <int G, int L>
+__host__ __device__ constexpr int min_blocks() {
+  return HQQ_MINB > 0 ? HQQ_MINB : (G / L < 32 ? 4 : (G == 32 ? 5 : 3));
+}
 
 __device__ __forceinline__ float round_even(float v) {
 #if HQQ_USE_FRND
@@ -135,6 +163,99 @@ __device__ __forceinline__ void load_group(const QArgs& a, int64_t g, int lane, 
   }
 }
 
+// axis 0 through shared memory: the block's NGB groups are NGB consecutive columns of one
+// row block (or of two, where the tile wraps), each G elements down its column. The block
+// reads the G element rows of the tile with 16-byte loads (consecutive threads take
+// consecutive 16-byte pieces of a row: coalesced), stores them to shared memory as a
+// [G][NGB] tile, and each lane then gathers its column's E elements from the tile.
+// Requires every 16-byte piece to lie in one row block: cols and NGB multiples of the
+// elements per 16 bytes (then n_groups and every tile start are too).
+template <int WDT>
+__host__ __device__ constexpr int elems_per_16B() { return WDT == kF32 ? 4 : 8; }
+
+template <int G, int NGB, int WDT>
+__device__ __forceinline__ void load_tile_axis0(const QArgs& a, int64_t g0, unsigned char* s_tile) {
+  constexpr int PERV = elems_per_16B<WDT>();
+  constexpr int ESZ = WDT == kF32 ? 4 : 2;
+  constexpr int CPR = NGB / PERV;  // 16-byte pieces per element row of the tile
+  const char* W = reinterpret_cast<const char*>(a.W);
+#pragma unroll 1
+  for (int k = threadIdx.x; k < G * CPR; k += kQBlock) {
+    const int j = k / CPR, i0 = (k - j * CPR) * PERV;
+    const int64_t gg = g0 + i0;
+    if (gg < a.n_groups) {
+      const int64_t rb = gg / a.cols, c = gg - rb * a.cols;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(W + ((rb * G + j) * a.cols + c) * ESZ));
+      *reinterpret_cast<uint4*>(s_tile + (j * NGB + i0) * ESZ) = v;
+    }
+  }
+}
+
+template <int G, int NGB, int E, int WDT>
+__device__ __forceinline__ void gather_tile_axis0(const unsigned char* s_tile, int gi, int lane,
+                                                  WRaw<WDT, E>& w) {
+  if constexpr (WDT == kF32) {
+    const uint32_t* t = reinterpret_cast<const uint32_t*>(s_tile);
+#pragma unroll
+    for (int j = 0; j < E; ++j) w.u[j] = t[(lane * E + j) * NGB + gi];
+  } else {
+    const unsigned short* t = reinterpret_cast<const unsigned short*>(s_tile);
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) {
+      const uint32_t lo = t[(lane * E + 2 * i) * NGB + gi];
+      const uint32_t hi = t[(lane * E + 2 * i + 1) * NGB + gi];
+      w.u[i] = lo | (hi << 16);
+    }
+  }
+}
+
+// axis 0 through shared memory, one warp at a time: a warp's 32/L groups are 32/L consecutive
+// columns of one row block (the tile start and 32/L are multiples of the elements per 16
+// bytes, and so is cols). The warp reads the G element rows of its columns with 16-byte loads
+// (32/L columns = 64/L bytes of a row: 4/L lanes per row, 8L rows per load instruction), stores
+// them to its own shared-memory region and, after a warp barrier only, each lane gathers its
+// E elements. Lane block l (rows l*E .. l*E+E-1) is stored after l spare rows, so that the L
+// lanes of a group read from disjoint banks.
+template <int G, int L, int WDT>
+__device__ __forceinline__ void load_warp_tile_axis0(const QArgs& a, int64_t gw0, int wl,
+                                                     unsigned char* s_w) {
+  constexpr int PERV = elems_per_16B<WDT>();
+  constexpr int ESZ = WDT == kF32 ? 4 : 2;
+  constexpr int WG = 32 / L, E = G / L;
+  constexpr int CPR = WG / PERV;  // 16-byte pieces per element row of the warp's columns
+  const char* W = reinterpret_cast<const char*>(a.W);
+#pragma unroll
+  for (int k = wl; k < G * CPR; k += 32) {
+    const int j = k / CPR, i0 = (k - j * CPR) * PERV;
+    const int64_t gg = gw0 + i0;
+    if (gg < a.n_groups) {
+      const int64_t rb = gg / a.cols, c = gg - rb * a.cols;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(W + ((rb * G + j) * a.cols + c) * ESZ));
+      *reinterpret_cast<uint4*>(s_w + ((j + j / E) * WG + i0) * ESZ) = v;
+    }
+  }
+}
+
+template <int G, int L, int WDT>
+__device__ __forceinline__ void gather_warp_tile_axis0(const unsigned char* s_w, int gi, int lane,
+                                                       WRaw<WDT, G / L>& w) {
+  constexpr int WG = 32 / L, E = G / L;
+  const int r0 = lane * E + lane;  // first stored row of this lane's block
+  if constexpr (WDT == kF32) {
+    const uint32_t* t = reinterpret_cast<const uint32_t*>(s_w);
+#pragma unroll
+    for (int j = 0; j < E; ++j) w.u[j] = t[(r0 + j) * WG + gi];
+  } else {
+    const unsigned short* t = reinterpret_cast<const unsigned short*>(s_w);
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) {
+      const uint32_t lo = t[(r0 + 2 * i) * WG + gi];
+      const uint32_t hi = t[(r0 + 2 * i + 1) * WG + gi];
+      w.u[i] = lo | (hi << 16);
+    }
+  }
+}
+
 // Exact shrinkage sum over this lane's elements, recomputed from memory (rare path).
 // Elements whose residual bound is below athr_lo have We == 0 exactly and are skipped.
 template <int G, int E, int AXIS, int WDT>
@@ -154,7 +275,9 @@ __device__ __noinline__ double shrink_sum_exact(const QArgs& a, int64_t g, int l
     const float r = __fsub_rn(w, __fmul_rn(__fsub_rn(q, z), step));
     const float ar = fabsf(r);
     if (!(ar > 0.0f)) continue;
-    const float t = powf(ar, pm1);
+    // |r|^(p-1) rounded once to fp32: the fp64 power, then one rounding (the correctly
+    // rounded fp32 value except within a few fp64 ulps of an fp32 rounding boundary)
+    const float t = __double2float_rn(pow((double)ar, (double)pm1));
     const float m = fmaxf(__fsub_rn(ar, __fmul_rn(t, inv_beta)), 0.0f);
     acc += (double)copysignf(m, r);
   }
@@ -218,6 +341,58 @@ __device__ __forceinline__ void evaluate(const float (&ws)[HQQ_STORE_WS ? E : 1]
   sq = qa[0] + qa[1];
 }
 
+// The same evaluation on pairs of elements (j, j+1): the fp32 adds of the definition and the
+// exponent product are lanes of add/mul.rn.f32x2, the residual's product is two scalar
+// multiplies (see below), so every rounding is that of the scalar code;
+// subtractions are additions of the negated operand (identical IEEE result), and
+// w - (q - z)*step is formed as w + (q - z)*(-step) (the product's rounding is symmetric).
+// The clamp, when needed, is applied per element before the rounding, as in the scalar path.
+template <int E, int WDT, bool CLAMP, bool P_ONE>
+__device__ __forceinline__ void evaluate_paired(const float (&ws)[HQQ_STORE_WS ? E : 1],
+                                                const WRaw<WDT, E>& w, float s, float z,
+                                                float step, float qmax, float pp, float& e,
+                                                float& sq) {
+  static_assert(E % 2 == 0, "pairs of elements");
+  const float2 z2 = make_float2(z, z), nz2 = make_float2(-z, -z);
+  const float2 pp2 = make_float2(pp, pp);
+  const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
+  const float2 nmagic2 = make_float2(-kRoundMagic, -kRoundMagic);
+  float2 ea[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 qa = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < E; j += 2) {
+    const float2 wsj = HQQ_STORE_WS ? make_float2(ws[j], ws[j + 1])
+                                    : fmul2_rn(make_float2(w.get(j), w.get(j + 1)),
+                                                 make_float2(s, s));
+    float2 v = fadd2_rn(wsj, z2);
+    if (CLAMP) v = make_float2(fminf(fmaxf(v.x, 0.0f), qmax), fminf(fmaxf(v.y, 0.0f), qmax));
+#if HQQ_USE_FRND
+    const float2 q = make_float2(rintf(v.x), rintf(v.y));
+#else
+    const float2 q = fadd2_rn(fadd2_rn(v, magic2), nmagic2);
+#endif
+    // the product stays two scalar multiplies: an f32x2 multiply feeding an f32x2 add was
+    // fused into one multiply-add by the code generator (one rounding instead of two), even
+    // with explicit .rn on both; __fmul_rn is never fused
+    const float2 d = fadd2_rn(q, nz2);
+    const float2 r = fadd2_rn(make_float2(w.get(j), w.get(j + 1)),
+                              make_float2(__fmul_rn(d.x, -step), __fmul_rn(d.y, -step)));
+    float2 term;
+    if (P_ONE) {
+      term = make_float2(fabsf(r.x), fabsf(r.y));
+    } else {
+      const float2 l = fmul2_rn(make_float2(lg2_approx(fabsf(r.x)), lg2_approx(fabsf(r.y))), pp2);
+      term = make_float2(ex2_approx(l.x), ex2_approx(l.y));
+    }
+    ea[(j >> 1) & 1] = fadd2_rn(ea[(j >> 1) & 1], term);
+    qa = fadd2_rn(qa, q);
+  }
+  // ea[0] holds the partial sums of j = 0, 1 (mod 4), ea[1] those of j = 2, 3: combined in
+  // the scalar path's order, so both variants return the same bits
+  e = __fadd_rn(__fadd_rn(ea[0].x, ea[0].y), __fadd_rn(ea[1].x, ea[1].y));
+  sq = qa.x + qa.y;
+}
+
 // The solver for the group this lane belongs to, from its raw weights in registers.
 // Returns the group's final codes (this lane's E of them), step and best zero.
 template <int G, int L, int AXIS, int WDT, bool STOP>
@@ -254,8 +429,13 @@ __device__ __forceinline__ void solve_group(const QArgs& a, int64_t g, int lane,
     acc = __dadd_rn(acc, f32_to_f64_exact(wsj));
   }
   if constexpr (L > 1) acc = group_sum_d<L>(acc, gmask);
-  const double S_ws = (double)(float)acc;  // rounded once to fp32
-  const double s_d = (double)s;
+  const float S_ws_f = __double2float_rn(acc);  // rounded once to fp32
+  // Without shrinkage (sum We = 0) the definition's update is fp32(fp64(sumQ - S_ws) / G).
+  // sumQ is an integer below 2^16 and S_ws an fp32 value; when S_ws is 0 or |S_ws| >= 2^-12
+  // both fit in 53 bits counted from the larger one's top bit down to S_ws's last bit, so the
+  // fp64 difference is exact and the update equals one fp32 subtraction (the exact difference
+  // rounded once) times the power of two 1/G (exact): no fp64 work on the common path.
+  const bool f32_update_exact = S_ws_f == 0.0f || fabsf(S_ws_f) >= 0x1p-12f;
   const float wsmin = __fmul_rn(mn, s), wsmax = __fmul_rn(mx, s);
 
   // ---- iterations
@@ -268,12 +448,22 @@ __device__ __forceinline__ void solve_group(const QArgs& a, int64_t g, int lane,
     const bool inside = __fadd_rn(wsmin, z) >= -0.5f && __fadd_rn(wsmax, z) < qmax + 0.5f;
     const bool clamp = __any_sync(wmask, !inside);
     float e, sq;
-    if (p_one) {
-      if (clamp) evaluate<E, WDT, true, true>(ws, w, s, z, step, qmax, pp, e, sq);
-      else evaluate<E, WDT, false, true>(ws, w, s, z, step, qmax, pp, e, sq);
+    if constexpr (HQQ_PAIRED && E % 2 == 0) {
+      if (p_one) {
+        if (clamp) evaluate_paired<E, WDT, true, true>(ws, w, s, z, step, qmax, pp, e, sq);
+        else evaluate_paired<E, WDT, false, true>(ws, w, s, z, step, qmax, pp, e, sq);
+      } else {
+        if (clamp) evaluate_paired<E, WDT, true, false>(ws, w, s, z, step, qmax, pp, e, sq);
+        else evaluate_paired<E, WDT, false, false>(ws, w, s, z, step, qmax, pp, e, sq);
+      }
     } else {
-      if (clamp) evaluate<E, WDT, true, false>(ws, w, s, z, step, qmax, pp, e, sq);
-      else evaluate<E, WDT, false, false>(ws, w, s, z, step, qmax, pp, e, sq);
+      if (p_one) {
+        if (clamp) evaluate<E, WDT, true, true>(ws, w, s, z, step, qmax, pp, e, sq);
+        else evaluate<E, WDT, false, true>(ws, w, s, z, step, qmax, pp, e, sq);
+      } else {
+        if (clamp) evaluate<E, WDT, true, false>(ws, w, s, z, step, qmax, pp, e, sq);
+        else evaluate<E, WDT, false, false>(ws, w, s, z, step, qmax, pp, e, sq);
+      }
     }
     if constexpr (L > 1) {
       e = group_sum<L>(e, gmask);
@@ -289,16 +479,25 @@ __device__ __forceinline__ void solve_group(const QArgs& a, int64_t g, int lane,
     // distance of the group's extreme scaled weight from the code range.
     const float hi = fmaxf(0.5f, fmaxf(-__fadd_rn(wsmin, z), __fsub_rn(__fadd_rn(wsmax, z), qmax)));
     const float bound = step * (hi * 1.001f + 1e-3f * (fabsf(z) + qmax + 1.0f));
-    double swe = 0.0;
     const bool no_shrink = bound < athr_lo;  // then also for every later update at this z
-    if (!no_shrink) {
-      swe = shrink_sum_exact<G, E, AXIS, WDT>(a, g, lane, s, step, z, __fdiv_rn(1.0f, beta), athr_lo);
-      if constexpr (L > 1) swe = group_sum_d<L>(swe, gmask);
-    }
     // Closed-form zero. Every lane computes it (a masked warp instruction costs the pipe as
     // much as a full one, so one lane computing and broadcasting would only add a shuffle).
-    const double num = __dadd_rn(__dsub_rn(small_int_f32_to_f64(sq), S_ws), __dmul_rn(s_d, swe));
-    const float znew = __double2float_rn(__dmul_rn(num, 1.0 / (double)G));  // G = 2^k: exact
+    float znew;
+    if (HQQ_F32_UPDATE && no_shrink && f32_update_exact) {
+      znew = __fmul_rn(__fsub_rn(sq, S_ws_f), 1.0f / (float)G);
+    } else {
+      // the definition's fp64 form z = fp32((sumQ - S_ws + s*sumWe) / G) (G = 2^k: the
+      // division is exact), with the exact shrinkage sum unless the bound rules it out
+      double swe = 0.0;
+      if (!no_shrink) {
+        swe = shrink_sum_exact<G, E, AXIS, WDT>(a, g, lane, s, step, z, __fdiv_rn(1.0f, beta),
+                                                athr_lo);
+        if constexpr (L > 1) swe = group_sum_d<L>(swe, gmask);
+      }
+      const double num = __dadd_rn(__dsub_rn(small_int_f32_to_f64(sq), (double)S_ws_f),
+                                   __dmul_rn((double)s, swe));
+      znew = __double2float_rn(__dmul_rn(num, 1.0 / (double)G));
+    }
     beta = __fmul_rn(beta, a.kappa);
     if constexpr (STOP) {
       // Fixed point: same zero, provably no shrinkage from here on, so every remaining
@@ -365,11 +564,18 @@ __device__ __forceinline__ int find_matrix(const QBatch<MAXB>& b, int64_t tile) 
 // each block's load / min-max / packing phases (a persistent grid-stride variant, where all
 // warps of an SM reach those phases together, measured 28 % slower).
 template <int G, int L, int AXIS, int WDT, bool PACK3, int MAXB, bool STOP>
-__global__ void __launch_bounds__(kQBlock, HQQ_MINB)
+__global__ void __launch_bounds__(kQBlock, min_blocks<G, L>())
     quantize_kernel(const __grid_constant__ QBatch<MAXB> batch) {
   constexpr int E = G / L;
   constexpr int NGB = kQBlock / L;  // groups per block
   __shared__ uint8_t s_codes[PACK3 ? NGB * G : 1];
+  constexpr bool kTile = HQQ_AXIS0_TILE == 1 && AXIS == 0 && NGB % elems_per_16B<WDT>() == 0;
+  constexpr bool kWTile =
+      HQQ_AXIS0_TILE == 2 && AXIS == 0 && (32 / L) % elems_per_16B<WDT>() == 0;
+  constexpr int kTileBytes = kTile ? G * NGB * (WDT == kF32 ? 4 : 2)
+                             : kWTile ? (kQBlock / 32) * (G + L) * (32 / L) * (WDT == kF32 ? 4 : 2)
+                                      : 16;
+  __shared__ __align__(16) unsigned char s_tile[kTileBytes];
 
   const int mi = MAXB == 1 ? 0 : find_matrix(batch, (int64_t)blockIdx.x);
   const int64_t tile = (int64_t)blockIdx.x - batch.tile_start[mi];
@@ -389,9 +595,27 @@ __global__ void __launch_bounds__(kQBlock, HQQ_MINB)
   const unsigned gmask = L == 1 ? 0u : (((1u << L) - 1u) << ((tid & 31) & ~(L - 1)));
   const float athr_lo = shrink_cutoff_lower_bound(a);
 
+  // axis 0: the tile paths when every 16-byte piece stays in one row block (block-uniform)
+  const bool tiled = (kTile || kWTile) && a.cols % elems_per_16B<WDT>() == 0;
+  constexpr int kWRegion = (G + L) * (32 / L) * (WDT == kF32 ? 4 : 2);  // per warp
+  unsigned char* s_w = s_tile + (tid / 32) * (kWTile ? kWRegion : 0);
+  if (tiled) {
+    if constexpr (kTile) {
+      load_tile_axis0<G, NGB, WDT>(a, tile * NGB, s_tile);
+      __syncthreads();
+    } else if constexpr (kWTile) {
+      load_warp_tile_axis0<G, L, WDT>(a, tile * NGB + (tid / 32) * (32 / L), tid & 31, s_w);
+      __syncwarp();
+    }
+  }
   if (valid) {
     WRaw<WDT, E> w;  // raw weights, resident for all evaluations
-    load_group<G, E, AXIS, WDT>(a, g, lane, w);
+    if (tiled) {
+      if constexpr (kTile) gather_tile_axis0<G, NGB, E, WDT>(s_tile, tid / L, lane, w);
+      if constexpr (kWTile) gather_warp_tile_axis0<G, L, WDT>(s_w, (tid & 31) / L, lane, w);
+    } else {
+      load_group<G, E, AXIS, WDT>(a, g, lane, w);
+    }
     uint32_t q[E];
     float step, zbest;
     solve_group<G, L, AXIS, WDT, STOP>(a, g, lane, gmask, wmask, athr_lo, w, q, step, zbest);
