@@ -39,7 +39,8 @@ sys.path.insert(0, HERE)
 
 METRIC = "HQQ quantize Gweights/s & % roofline (HBM|SFU), 7B-shaped bf16 4-bit g64"
 UNIT = "Gweights/s"
-MUFU_PER_CLK_PER_SM = 16          # lg2/ex2 issue rate of the B200 SFU (probed: 15.9)
+MUFU_PER_CLK_PER_SM = 16          # lg2/ex2 issue rate of the B200 SFU (probed: 15.9 with
+                                  # bench_probes/probe.py sfu)
 N_SM = 148
 SM_MAX_MHZ = 1965.0
 
@@ -197,6 +198,8 @@ def run_ours(args, rank, world, dev):
         if ev is not None:
             ev[0][1].record(stream)
         hqq.hqq_dequantize_batched(outs, shapes, params, W_out=deqs, batch=dbatch, stream=stream)
+        if ev is not None:
+            ev[0][2].record(stream)
 
     def barrier():
         if world > 1:
@@ -207,7 +210,7 @@ def run_ours(args, rank, world, dev):
         step()
     barrier()
     n_q = len(mats) if args.per_matrix else 1  # solver launches per step
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_q)]
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_q)]
            for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
@@ -219,6 +222,7 @@ def run_ours(args, rank, world, dev):
         barrier()
     ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     q_ms = [e[0].elapsed_time(e[1]) for ev in evs for e in ev]
+    dq_ms = None if args.per_matrix else [ev[0][1].elapsed_time(ev[0][2]) for ev in evs]
     ms_step = ms_total / args.steps
     # weak: every rank did a whole model; strong (--shard): the ranks shared one model
     total_weights = workloads.llama7b_model_4b().weights if args.shard else world * n_w
@@ -250,7 +254,8 @@ def run_ours(args, rank, world, dev):
                                          else "1 batched solver + 1 batched dequantize"),
                    "l2": "inputs 13 GB > 126 MB L2, no flush",
                    "quantize_share_of_step": round(quant_share, 4),
-                   "quantize_Gweights_per_s": round(n_w / (sum(q_ms) / args.steps * 1e-3) / 1e9, 3)},
+                   "quantize_Gweights_per_s": round(n_w / (sum(q_ms) / args.steps * 1e-3) / 1e9, 3),
+                   "dequantize": _dequant_figures(dq_ms, n_w, pk)},
         "roofline": {"bound": "alu", "kernel": "quantize_kernel (MUFU lg2+ex2)",
                      "achieved": round(achieved, 4), "peak": round(peak, 4), "unit": "Top/s (MUFU)",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -267,15 +272,31 @@ def run_ours(args, rank, world, dev):
         res["fixed_point_stop"] = run_fixed_point(hqq, wl, Ws, outs, deqs, params, shapes,
                                                   stream, args)
     if rank == 0 and not args.no_e2e:
-        res["e2e"] = run_e2e(hqq, wl, Ws, outs, dev, args)
+        res["e2e"] = run_e2e(hqq, wl, Ws, outs, params, dev, args)
     if rank == 0 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(wl, Ws, args.cpu_seconds)
     if rank == 0 and not args.no_linear:
         del Ws, outs, deqs, qbatch, dbatch
         torch.cuda.empty_cache()
+        if not args.no_configs:
+            res["configs"] = configs_table(reps=max(3, min(args.steps, 10)))
         res["w4a16_linear"] = run_linear(hqq, dev, args)
         res["mxfp4_weightonly"] = run_mxfp4(hqq, dev, args)
     return res
+
+
+def _dequant_figures(dq_ms, n_w, pk):
+    """The batched dequantize launch of the step: average duration (CUDA events around it on
+    the launch stream), algorithmic GB/s (2.5625 B per weight: read 0.5 B of codes and 4 B of
+    bf16 scale/zero per 64 weights, write 2 B) and the fraction of the measured HBM copy
+    bandwidth."""
+    if not dq_ms:
+        return None
+    ms = sum(dq_ms) / len(dq_ms)
+    gbs = 2.5625 * n_w / (ms * 1e-3) / 1e9
+    return {"kernel": "dequant4_axis1_kernel (batched)", "avg_launch_ms": round(ms, 4),
+            "GB_per_s": round(gbs, 1), "hbm_frac": round(gbs / pk["hbm_gbs"], 4),
+            "algorithmic": "2.5625 B/weight"}
 
 
 def solver_source_digest() -> str:
@@ -539,65 +560,89 @@ def run_mxfp4(hqq, dev, args):
             "gpu_launches": 2 * args.steps}
 
 
-def run_e2e(hqq, wl, Ws, outs, dev, args):
-    """Same metric through the public API with host buffers: every step copies each weight
-    from pinned host memory, quantizes and dequantizes it, and reads the packed codes and
-    scale/zero back into pinned host memory; copies overlap compute on separate streams."""
+def run_e2e(hqq, wl, Ws, outs, params, dev, args):
+    """Same metric through the public API with host buffers, on the batched calls the
+    headline uses: every step copies each weight from pinned host memory, quantizes and
+    dequantizes it, and reads the quantized model (packed codes, scale, zero) back into pinned
+    host memory. The model goes through in chunks of one decoder block (7 matrices: one
+    hqq_quantize_batched and one hqq_dequantize_batched call each), so that the host-to-device
+    copy of block b+1, the kernels of block b and the device-to-host copy of block b-1 overlap
+    on three streams; three staging slots on the device hold the blocks in flight."""
     mats = wl.matrices
     host_W = [torch.empty_like(W, device="cpu", pin_memory=True).copy_(W) for W in Ws]
     host_out = [tuple(torch.empty_like(t, device="cpu", pin_memory=True) for t in o)
                 for o in outs]
-    comp = torch.cuda.Stream(dev)
-    h2d = torch.cuda.Stream(dev)
-    d2h = torch.cuda.Stream(dev)
-    n_stage = 3
-    big = max(m.rows * m.cols for m in mats)
-    stage = [torch.empty(big, dtype=torch.bfloat16, device=dev) for _ in range(n_stage)]
-    stage_free = [torch.cuda.Event() for _ in range(n_stage)]
-    deq = torch.empty(big, dtype=torch.bfloat16, device=dev)
+    comp, h2d, d2h = (torch.cuda.Stream(dev) for _ in range(3))
+    per_chunk = 7
+    chunks = [list(range(i, min(i + per_chunk, len(mats)))) for i in range(0, len(mats), per_chunk)]
+    n_slot = 3
+    slot_elems = max(sum(mats[i].numel for i in c) for c in chunks)
+    slot_in = [torch.empty(slot_elems, dtype=torch.bfloat16, device=dev) for _ in range(n_slot)]
+    slot_deq = [torch.empty(slot_elems, dtype=torch.bfloat16, device=dev) for _ in range(n_slot)]
+    views, qb, db = [], [], []
+    for c_i, c in enumerate(chunks):
+        s, off, wv, dv = c_i % n_slot, 0, [], []
+        for i in c:
+            m = mats[i]
+            wv.append(slot_in[s][off:off + m.numel].view(m.rows, m.cols))
+            dv.append(slot_deq[s][off:off + m.numel].view(m.rows, m.cols))
+            off += m.numel
+        views.append((wv, dv))
+        qb.append(hqq.matrix_batch(wv, [outs[i] for i in c]))
+        db.append(hqq.matrix_batch(dv, [outs[i] for i in c]))
+    slot_free = [torch.cuda.Event() for _ in range(n_slot)]
+    for e in slot_free:
+        e.record(comp)
     h2d_bytes = sum(W.numel() * W.element_size() for W in host_W)
     d2h_bytes = sum(sum(t.numel() * t.element_size() for t in o) for o in host_out)
+    launches = 0
 
     def step():
-        out_ready = []
-        for i, m in enumerate(mats):
-            b = i % n_stage
-            buf = stage[b][: m.rows * m.cols].view(m.rows, m.cols)
-            h2d.wait_event(stage_free[b])
+        nonlocal launches
+        for c_i, c in enumerate(chunks):
+            s = c_i % n_slot
+            wv, dv = views[c_i]
+            h2d.wait_event(slot_free[s])
             with torch.cuda.stream(h2d):
-                buf.copy_(host_W[i], non_blocking=True)
+                for i, buf in zip(c, wv):
+                    buf.copy_(host_W[i], non_blocking=True)
                 loaded = torch.cuda.Event()
                 loaded.record(h2d)
             comp.wait_event(loaded)
-            p, s, z = outs[i]
-            hqq.hqq_quantize(buf, m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0, m.kappa,
-                             Wq_packed=p, scale=s, zero=z, stream=comp)
-            hqq.hqq_dequantize(p, s, z, m.rows, m.cols, m.nbits, m.group_size, m.axis,
-                               out=deq[: m.rows * m.cols].view(m.rows, m.cols), stream=comp)
-            stage_free[b].record(comp)
+            sub_outs = [outs[i] for i in c]
+            hqq.hqq_quantize_batched(wv, params, outs=sub_outs, batch=qb[c_i], stream=comp)
+            hqq.hqq_dequantize_batched(sub_outs, [tuple(v.shape) for v in dv], params,
+                                       W_out=dv, batch=db[c_i], stream=comp)
+            launches += 2
+            slot_free[s].record(comp)
             done = torch.cuda.Event()
             done.record(comp)
             d2h.wait_event(done)
             with torch.cuda.stream(d2h):
-                for src, dst in zip(outs[i], host_out[i]):
-                    dst.copy_(src, non_blocking=True)
+                for i in c:
+                    for src, dst in zip(outs[i], host_out[i]):
+                        dst.copy_(src, non_blocking=True)
         d2h.synchronize()
         comp.synchronize()
 
     for _ in range(2):
         step()
     torch.cuda.synchronize()
-    steps = max(1, min(args.steps, 3))
+    launches = 0
     t = time.perf_counter()
-    for _ in range(steps):
+    for _ in range(args.steps):
         step()
     torch.cuda.synchronize()
-    sec = (time.perf_counter() - t) / steps
+    sec = (time.perf_counter() - t) / args.steps
     return {"value": round(wl.weights / sec / 1e9, 3), "unit": UNIT,
             "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
-            "ms_per_step": round(sec * 1e3, 2), "steps": steps,
-            "how": "pinned host W -> device (stream 1), quantize+dequantize (stream 2), "
-                   "packed+scale+zero -> pinned host (stream 3); wall clock with device sync"}
+            "ms_per_step": round(sec * 1e3, 2), "steps": args.steps,
+            "gpu_launches": launches,
+            "how": "per decoder block (7 matrices): pinned host W -> device (stream 1); "
+                   "hqq_quantize_batched + hqq_dequantize_batched (stream 2); the quantized "
+                   "model (packed codes, scale, zero; 3.64 GB) -> pinned host (stream 3). "
+                   "The dequantized weights stay on the device (read back: none). Wall clock "
+                   "with device synchronisation around the timed steps."}
 
 
 def cpu_baseline(wl, Ws, seconds: float, impl_line=False):
@@ -657,73 +702,6 @@ def run_reference(args, rank, world):
                              "sample": desc},
             "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
-
-
-def probe_sfu():
-    """Measured lg2/ex2 issue rate per SM per clock (the solver's bound), from the probe
-    kernel in csrc/hqq_probe.cu; clocks sampled meanwhile."""
-    import ctypes
-    L = ctypes.CDLL(os.path.join(HERE, "calibration_free_weight_hqq_b200", "libhqq_probe.so"))
-    L.hqq_probe_sfu.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
-                                ctypes.c_int, ctypes.c_void_p]
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    res = {"probe": "sfu", "sms": sms}
-    with ClockSampler(0) as clk:
-        for op, per, name in ((0, 1, "ex2"), (1, 1, "lg2"), (2, 2, "lg2+ex2")):
-            blocks, threads, iters = sms * 8, 256, 4096
-            out = torch.empty(blocks * threads, device="cuda")
-            st = torch.cuda.current_stream()
-            for _ in range(2):
-                assert L.hqq_probe_sfu(op, out.data_ptr(), blocks, threads, iters, st.cuda_stream) == 0
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(st)
-            L.hqq_probe_sfu(op, out.data_ptr(), blocks, threads, iters, st.cuda_stream)
-            e1.record(st)
-            torch.cuda.synchronize()
-            ms = e0.elapsed_time(e1)
-            ops = blocks * threads * iters * 8 * per
-            res[name] = {"ms": round(ms, 3), "ops_per_s": ops / (ms * 1e-3)}
-    c = clk.summary()
-    res["clocks"] = c
-    # The probe runs for milliseconds, shorter than the 200 ms clock sampling, so the rate
-    # is normalised at the maximum SM clock (the clock held under the bench's sustained load).
-    mhz = c.get("sm_max_mhz") or SM_MAX_MHZ
-    res["normalised_at_mhz"] = mhz
-    for name in ("ex2", "lg2", "lg2+ex2"):
-        res[name]["per_clk_per_sm"] = round(res[name]["ops_per_s"] / sms / (mhz * 1e6), 2)
-    return res
-
-
-def probe_hbm(gib: float = 1.0):
-    """HBM bandwidth for read-only, write-only and copy traffic (16-byte accesses, grid of
-    SMs x 8 blocks of 256 threads), on a buffer of `gib` GiB (far above L2)."""
-    import ctypes
-    L = ctypes.CDLL(os.path.join(HERE, "calibration_free_weight_hqq_b200", "libhqq_probe.so"))
-    L.hqq_probe_hbm.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
-                                ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    blocks, threads = sms * 8, 256
-    nbytes = int(gib * (1 << 30)) // 16 * 16
-    a = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
-    b = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
-    sink = torch.empty(blocks * threads, dtype=torch.int32, device="cuda")
-    st = torch.cuda.current_stream()
-    res = {"probe": "hbm", "bytes": nbytes}
-    for op, name, moved in ((0, "write", nbytes), (1, "read", nbytes), (2, "copy", 2 * nbytes)):
-        dst = sink if op == 1 else b
-        for _ in range(3):
-            assert L.hqq_probe_hbm(op, a.data_ptr(), dst.data_ptr(), nbytes, blocks, threads,
-                                   st.cuda_stream) == 0
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(st)
-        for _ in range(10):
-            L.hqq_probe_hbm(op, a.data_ptr(), dst.data_ptr(), nbytes, blocks, threads,
-                            st.cuda_stream)
-        e1.record(st)
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / 10
-        res[name] = {"ms": round(ms, 4), "GB_per_s": round(moved / ms / 1e6, 1)}
-    return res
 
 
 def single_linear(reps: int = 10, M: int = 4096):
@@ -927,24 +905,16 @@ def main():
     ap.add_argument("--no-linear", action="store_true",
                     help="skip the fused 4-bit linear-layer measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--probe-sfu", action="store_true",
-                    help="measure the lg2/ex2 issue rate behind the roofline peak and exit")
-    ap.add_argument("--probe-hbm", action="store_true",
-                    help="measure HBM read-only, write-only and copy bandwidth and exit")
     ap.add_argument("--configs", action="store_true",
-                    help="quantize/dequantize throughput of the four smaller configurations")
+                    help="print only the four smaller configurations' lines and exit")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="leave the four smaller configurations out of the JSON line")
     ap.add_argument("--mixed", action="store_true",
                     help="whole model with per-layer configurations (8/4/2 bits) and exit")
     ap.add_argument("--single", choices=["quantize", "dequantize", "linear", "decode"],
                     help="time one [16384,8192] matrix, one 4096^3 linear layer, or one "
                          "4096x4096 layer at 16 tokens (the profiling cases), and exit")
     args = ap.parse_args()
-    if args.probe_sfu:
-        print(json.dumps(probe_sfu()), flush=True)
-        return
-    if args.probe_hbm:
-        print(json.dumps(probe_hbm()), flush=True)
-        return
     if args.configs:
         for line in configs_table():
             print(json.dumps(line), flush=True)

@@ -1,7 +1,8 @@
 // hqq_probe.cu - throughput probes behind the rooflines: the special-function unit (MUFU
 // lg2/ex2, which bounds the HQQ solver) and HBM read-only / write-only / copy bandwidth (the
 // dequantizer writes 4 bytes for every byte it reads at 4 bits). Built into a separate
-// library (libhqq_probe.so), not the quantization ABI; bench.py --probe-sfu / --probe-hbm.
+// library (bench_probes/libhqq_probe.so), not the quantization ABI; run by
+// `python bench_probes/probe.py sfu` / `python bench_probes/probe.py hbm`.
 //
 // Every thread runs 8 independent dependency chains of approximate lg2/ex2 (and nothing
 // else but one FADD/FMUL per step), so the SFU issue rate, not latency, limits the kernel.

@@ -17,10 +17,9 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 BUILD_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libhqq_b200.so")
-PROBE_LIB = os.path.join(HERE, "libhqq_probe.so")  # SFU throughput probe used by bench.py
 SOURCES = ["hqq_abi.cu", "hqq_quantize.cu", "hqq_quantize_stop.cu", "hqq_dequantize.cu",
            "hqq_noalloc.cu", "hqq_gemm.cu", "hqq_mx.cu"]
-HEADERS = ["hqq_device.cuh", "hqq_kernels.h", "hqq_quantize_impl.cuh"]
+HEADERS = ["hqq_device.cuh", "hqq_kernels.h", "hqq_quantize_impl.cuh", "hqq_abi_internal.h"]
 PUBLIC_HEADER = os.path.join(ROOT, "include", "hqq", "hqq.h")
 
 NVCC_FLAGS = [
@@ -70,12 +69,6 @@ def build(force: bool = False, verbose: bool = False) -> str:
         subprocess.check_call([nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
                                *objs, "-o", tmp])
         os.replace(tmp, LIB)
-    probe_src = os.path.join(CSRC, "hqq_probe.cu")
-    if force or _stale(PROBE_LIB, [probe_src, __file__]):
-        tmp = PROBE_LIB + ".tmp.%d" % os.getpid()
-        flags = [f for f in NVCC_FLAGS if f not in ("-Xptxas", "-v", "-fmad=false")]
-        subprocess.check_call([nvcc(), *flags, "-shared", probe_src, "-o", tmp])
-        os.replace(tmp, PROBE_LIB)
     return LIB
 
 
