@@ -860,19 +860,31 @@ def run_mixed_model(args):
             "ms_per_step": round(ms, 3), "launches_per_step": 2 * groups, "steps": args.steps}
 
 
+# The single-matrix profiling cases: (rows, cols, dtype, nbits, group_size, axis). Each input
+# is larger than the 126 MB L2 except the [4096, 1024] fp16 matrix of the single-layer workload.
+SINGLE_CASES = {
+    "quantize": (16384, 8192, "bf16", 4, 64, 1),
+    "dequantize": (16384, 8192, "bf16", 4, 64, 1),
+    "quantize_2b_g16_axis0": (16384, 8192, "bf16", 2, 16, 0),
+    "quantize_1b_g32": (16384, 8192, "bf16", 1, 32, 1),
+    "quantize_3b_g64": (16384, 8192, "bf16", 3, 64, 1),
+    "quantize_fp16_4096x1024": (4096, 1024, "f16", 4, 64, 1),
+}
+
+
 def single(kind: str, reps: int = 10):
-    """One [16384, 8192] bf16 matrix (134M weights, 268 MB: larger than L2), 4-bit g64:
-    time `reps` solver or dequantize launches after warm-up (the small case the ncu
-    captures in profiles/ use)."""
+    """One matrix of SINGLE_CASES[kind]: time `reps` solver or dequantize launches after
+    warm-up (the cases the ncu captures in profiles/ use)."""
     import calibration_free_weight_hqq_b200 as hqq
     from calibration_free_weight_hqq_b200 import synthetic
-    rows, cols = 16384, 8192
-    W = synthetic.weight(rows, cols, seed=5, dtype=torch.bfloat16, device="cuda")
-    pk, s, z = hqq.hqq_quantize(W, 4, 64, 1)
+    rows, cols, dt, nbits, G, axis = SINGLE_CASES[kind]
+    dtype = torch.float16 if dt == "f16" else torch.bfloat16
+    W = synthetic.weight(rows, cols, seed=5, dtype=dtype, device="cuda")
+    pk, s, z = hqq.hqq_quantize(W, nbits, G, axis)
     D = torch.empty_like(W)
-    run = (lambda: hqq.hqq_quantize(W, 4, 64, 1, Wq_packed=pk, scale=s, zero=z)) \
-        if kind == "quantize" else \
-        (lambda: hqq.hqq_dequantize(pk, s, z, rows, cols, 4, 64, 1, out=D))
+    run = (lambda: hqq.hqq_dequantize(pk, s, z, rows, cols, nbits, G, axis, out=D)) \
+        if kind == "dequantize" else \
+        (lambda: hqq.hqq_quantize(W, nbits, G, axis, Wq_packed=pk, scale=s, zero=z))
     for _ in range(2):
         run()
     torch.cuda.synchronize()
@@ -884,9 +896,10 @@ def single(kind: str, reps: int = 10):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
     n = rows * cols
-    return {"single": kind, "shape": [rows, cols], "ms": round(ms, 4),
-            "Gweights_per_s": round(n / ms / 1e6, 2),
-            "GB_per_s_algorithmic": round(n * 2.5625 / ms / 1e6, 1)}
+    mufu = 2 * 21 * n / (ms * 1e-3) / (MUFU_PER_CLK_PER_SM * N_SM * SM_MAX_MHZ * 1e6)
+    return {"single": kind, "shape": [rows, cols], "nbits": nbits, "group_size": G,
+            "axis": axis, "ms": round(ms, 4), "Gweights_per_s": round(n / ms / 1e6, 2),
+            "mufu_frac": round(mufu, 4) if kind != "dequantize" else None}
 
 
 def main():
@@ -911,9 +924,9 @@ def main():
                     help="leave the four smaller configurations out of the JSON line")
     ap.add_argument("--mixed", action="store_true",
                     help="whole model with per-layer configurations (8/4/2 bits) and exit")
-    ap.add_argument("--single", choices=["quantize", "dequantize", "linear", "decode"],
-                    help="time one [16384,8192] matrix, one 4096^3 linear layer, or one "
-                         "4096x4096 layer at 16 tokens (the profiling cases), and exit")
+    ap.add_argument("--single", choices=sorted(SINGLE_CASES) + ["linear", "decode"],
+                    help="time one matrix of a profiling case (SINGLE_CASES), one 4096^3 "
+                         "linear layer, or one 4096x4096 layer at 16 tokens, and exit")
     args = ap.parse_args()
     if args.configs:
         for line in configs_table():

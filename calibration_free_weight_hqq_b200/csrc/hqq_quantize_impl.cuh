@@ -46,13 +46,11 @@ constexpr int kQBlock = 160;  // 5 warps; kQBlock*E codes per block is a multipl
 
 // Resident blocks per SM the register budget is sized for (measured on B200, every shape of
 // the shipped workloads): with 32 elements per lane the raw and scaled weights take 48
-// registers, and 3 blocks (128 registers a thread, no spills) ran faster than 4 (96, spills)
-// for groups of 64 and more; groups of 32 (one lane each) ran fastest with 5 blocks, whose
-// extra warps hide the lanes that take the exact shrinkage path; with 16 or fewer elements
-// per lane 4 blocks fit without spills.
+// registers, and 3 blocks (128 registers a thread, no spills) ran faster than 4 or 5 (96 or
+// 72 registers, spills); with 16 or fewer elements per lane 4 blocks fit without spills.
 template <int G, int L>
 __host__ __device__ constexpr int min_blocks() {
-  return HQQ_MINB > 0 ? HQQ_MINB : (G / L < 32 ? 4 : (G == 32 ? 5 : 3));
+  return HQQ_MINB > 0 ? HQQ_MINB : (G / L < 32 ? 4 : 3);
 }
 
 __device__ __forceinline__ float round_even(float v) {
@@ -62,6 +60,19 @@ __device__ __forceinline__ float round_even(float v) {
   return rint_magic(v);
 #endif
 }
+
+// Shrinkage cut-offs of the updates: We = max(|r| - |r|^(p-1)/beta_k, 0) is nonzero only
+// where |r|^(2-p) > 1/beta_k. cut[k] = (1/beta_k)^(1/(2-p)) * (1 - 1e-5) for update k, with
+// beta_k and 1/beta_k formed by the same fp32 operations as the kernel's, evaluated on the host
+// in fp64 and rounded down to fp32. Below cut[k] every rounded |r|^(p-1)/beta_k still exceeds
+// |r| (the margin covers the power's, the product's and the difference's roundings), so We is
+// exactly 0. Updates past the table use cut_min, the last update's cut-off (beta only grows,
+// so it is the smallest), which also decides when a group can never shrink again.
+constexpr int kCutTable = 64;
+struct ShrinkCut {
+  float cut[kCutTable];
+  float cut_min;
+};
 
 struct QArgs {
   const void* W;
@@ -257,11 +268,12 @@ __device__ __forceinline__ void gather_warp_tile_axis0(const unsigned char* s_w,
 }
 
 // Exact shrinkage sum over this lane's elements, recomputed from memory (rare path).
-// Elements whose residual bound is below athr_lo have We == 0 exactly and are skipped.
+// `cut` is this update's cut-off with its rounding margin (ShrinkCut): elements whose
+// residual is below it have We == 0 exactly and are skipped before the power.
 template <int G, int E, int AXIS, int WDT>
 __device__ __noinline__ double shrink_sum_exact(const QArgs& a, int64_t g, int lane, float s,
                                                 float step, float z, float inv_beta,
-                                                float athr_lo) {
+                                                float cut) {
   const float slack = 1e-3f * (fabsf(z) + a.qmax + 1.0f);
   const float pm1 = a.p - 1.0f;
   double acc = 0.0;
@@ -271,10 +283,10 @@ __device__ __noinline__ double shrink_sum_exact(const QArgs& a, int64_t g, int l
     const float v = __fadd_rn(__fmul_rn(w, s), z);
     const float q = fminf(fmaxf(rintf(v), 0.0f), a.qmax);
     const float d = __fsub_rn(v, q);
-    if (step * (fabsf(d) * 1.001f + slack) < athr_lo) continue;
+    if (step * (fabsf(d) * 1.001f + slack) < cut) continue;
     const float r = __fsub_rn(w, __fmul_rn(__fsub_rn(q, z), step));
     const float ar = fabsf(r);
-    if (!(ar > 0.0f)) continue;
+    if (!(ar >= cut)) continue;  // below the cut-off (or zero): We == 0 exactly
     // |r|^(p-1) rounded once to fp32: the fp64 power, then one rounding (the correctly
     // rounded fp32 value except within a few fp64 ulps of an fp32 rounding boundary)
     const float t = __double2float_rn(pow((double)ar, (double)pm1));
@@ -320,13 +332,14 @@ __device__ __forceinline__ void store_codes(uint8_t* packed, int64_t code0, cons
 
 // One evaluation of candidate zero z over this lane's elements: the lp error (four
 // partial sums) and the code sum.
-template <int E, int WDT, bool CLAMP, bool P_ONE>
+template <int E, int WDT, bool CLAMP, bool P_ONE, bool TRACK>
 __device__ __forceinline__ void evaluate(const float (&ws)[HQQ_STORE_WS ? E : 1],
                                          const WRaw<WDT, E>& w, float s,
                                          float z, float step, float qmax, float pp, float& e,
-                                         float& sq) {
+                                         float& sq, float& rmax) {
   float ea[4] = {0.f, 0.f, 0.f, 0.f};
   float qa[2] = {0.f, 0.f};
+  float rm = 0.0f;
 #pragma unroll
   for (int j = 0; j < E; ++j) {
     const float wsj = HQQ_STORE_WS ? ws[j] : __fmul_rn(w.get(j), s);
@@ -336,9 +349,11 @@ __device__ __forceinline__ void evaluate(const float (&ws)[HQQ_STORE_WS ? E : 1]
     const float term = P_ONE ? fabsf(r) : ex2_approx(__fmul_rn(pp, lg2_approx(fabsf(r))));
     ea[j & 3] = __fadd_rn(ea[j & 3], term);
     qa[j & 1] += q;
+    if (TRACK) rm = fmaxf(rm, fabsf(r));
   }
   e = __fadd_rn(__fadd_rn(ea[0], ea[1]), __fadd_rn(ea[2], ea[3]));
   sq = qa[0] + qa[1];
+  rmax = rm;
 }
 
 // The same evaluation on pairs of elements (j, j+1): the fp32 adds of the definition and the
@@ -347,11 +362,11 @@ __device__ __forceinline__ void evaluate(const float (&ws)[HQQ_STORE_WS ? E : 1]
 // subtractions are additions of the negated operand (identical IEEE result), and
 // w - (q - z)*step is formed as w + (q - z)*(-step) (the product's rounding is symmetric).
 // The clamp, when needed, is applied per element before the rounding, as in the scalar path.
-template <int E, int WDT, bool CLAMP, bool P_ONE>
+template <int E, int WDT, bool CLAMP, bool P_ONE, bool TRACK>
 __device__ __forceinline__ void evaluate_paired(const float (&ws)[HQQ_STORE_WS ? E : 1],
                                                 const WRaw<WDT, E>& w, float s, float z,
                                                 float step, float qmax, float pp, float& e,
-                                                float& sq) {
+                                                float& sq, float& rmax) {
   static_assert(E % 2 == 0, "pairs of elements");
   const float2 z2 = make_float2(z, z), nz2 = make_float2(-z, -z);
   const float2 pp2 = make_float2(pp, pp);
@@ -359,6 +374,7 @@ __device__ __forceinline__ void evaluate_paired(const float (&ws)[HQQ_STORE_WS ?
   const float2 nmagic2 = make_float2(-kRoundMagic, -kRoundMagic);
   float2 ea[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   float2 qa = make_float2(0.f, 0.f);
+  float rm0 = 0.0f, rm1 = 0.0f;
 #pragma unroll
   for (int j = 0; j < E; j += 2) {
     const float2 wsj = HQQ_STORE_WS ? make_float2(ws[j], ws[j + 1])
@@ -386,18 +402,48 @@ __device__ __forceinline__ void evaluate_paired(const float (&ws)[HQQ_STORE_WS ?
     }
     ea[(j >> 1) & 1] = fadd2_rn(ea[(j >> 1) & 1], term);
     qa = fadd2_rn(qa, q);
+    if (TRACK) {
+      rm0 = fmaxf(rm0, fabsf(r.x));
+      rm1 = fmaxf(rm1, fabsf(r.y));
+    }
   }
   // ea[0] holds the partial sums of j = 0, 1 (mod 4), ea[1] those of j = 2, 3: combined in
   // the scalar path's order, so both variants return the same bits
   e = __fadd_rn(__fadd_rn(ea[0].x, ea[0].y), __fadd_rn(ea[1].x, ea[1].y));
   sq = qa.x + qa.y;
+  rmax = fmaxf(rm0, rm1);
+}
+
+// One evaluation, dispatched on the warp-uniform flags to the compiled variants.
+template <int E, int WDT, bool TRACK>
+__device__ __forceinline__ void evaluate_any(const float (&ws)[HQQ_STORE_WS ? E : 1],
+                                             const WRaw<WDT, E>& w, float s, float z, float step,
+                                             float qmax, float pp, bool p_one, bool clamp,
+                                             float& e, float& sq, float& rmax) {
+  if constexpr (HQQ_PAIRED && E % 2 == 0) {
+    if (p_one) {
+      if (clamp) evaluate_paired<E, WDT, true, true, TRACK>(ws, w, s, z, step, qmax, pp, e, sq, rmax);
+      else evaluate_paired<E, WDT, false, true, TRACK>(ws, w, s, z, step, qmax, pp, e, sq, rmax);
+    } else {
+      if (clamp) evaluate_paired<E, WDT, true, false, TRACK>(ws, w, s, z, step, qmax, pp, e, sq, rmax);
+      else evaluate_paired<E, WDT, false, false, TRACK>(ws, w, s, z, step, qmax, pp, e, sq, rmax);
+    }
+  } else {
+    if (p_one) {
+      if (clamp) evaluate<E, WDT, true, true, TRACK>(ws, w, s, z, step, qmax, pp, e, sq, rmax);
+      else evaluate<E, WDT, false, true, TRACK>(ws, w, s, z, step, qmax, pp, e, sq, rmax);
+    } else {
+      if (clamp) evaluate<E, WDT, true, false, TRACK>(ws, w, s, z, step, qmax, pp, e, sq, rmax);
+      else evaluate<E, WDT, false, false, TRACK>(ws, w, s, z, step, qmax, pp, e, sq, rmax);
+    }
+  }
 }
 
 // The solver for the group this lane belongs to, from its raw weights in registers.
 // Returns the group's final codes (this lane's E of them), step and best zero.
 template <int G, int L, int AXIS, int WDT, bool STOP>
 __device__ __forceinline__ void solve_group(const QArgs& a, int64_t g, int lane, unsigned gmask,
-                                            unsigned wmask, float athr_lo,
+                                            unsigned wmask, const ShrinkCut& sc,
                                             const WRaw<WDT, G / L>& w, uint32_t (&q)[G / L],
                                             float& step_out, float& zbest_out) {
   constexpr int E = G / L;
@@ -447,24 +493,19 @@ __device__ __forceinline__ void solve_group(const QArgs& a, int64_t g, int lane,
     // rint(v) >= 0 for v >= -0.5 and rint(v) <= qmax for v < qmax + 0.5.
     const bool inside = __fadd_rn(wsmin, z) >= -0.5f && __fadd_rn(wsmax, z) < qmax + 0.5f;
     const bool clamp = __any_sync(wmask, !inside);
-    float e, sq;
-    if constexpr (HQQ_PAIRED && E % 2 == 0) {
-      if (p_one) {
-        if (clamp) evaluate_paired<E, WDT, true, true>(ws, w, s, z, step, qmax, pp, e, sq);
-        else evaluate_paired<E, WDT, false, true>(ws, w, s, z, step, qmax, pp, e, sq);
-      } else {
-        if (clamp) evaluate_paired<E, WDT, true, false>(ws, w, s, z, step, qmax, pp, e, sq);
-        else evaluate_paired<E, WDT, false, false>(ws, w, s, z, step, qmax, pp, e, sq);
-      }
-    } else {
-      if (p_one) {
-        if (clamp) evaluate<E, WDT, true, true>(ws, w, s, z, step, qmax, pp, e, sq);
-        else evaluate<E, WDT, false, true>(ws, w, s, z, step, qmax, pp, e, sq);
-      } else {
-        if (clamp) evaluate<E, WDT, true, false>(ws, w, s, z, step, qmax, pp, e, sq);
-        else evaluate<E, WDT, false, false>(ws, w, s, z, step, qmax, pp, e, sq);
-      }
-    }
+    // Bound on max_j |r_j| at this zero: unclamped codes leave |v - Q| <= 1/2, clamped ones at
+    // most the distance of the group's extreme scaled weight from the code range.
+    const float hi = fmaxf(0.5f, fmaxf(-__fadd_rn(wsmin, z), __fsub_rn(__fadd_rn(wsmax, z), qmax)));
+    const float bound = step * (hi * 1.001f + 1e-3f * (fabsf(z) + qmax + 1.0f));
+    const float cutk = k < kCutTable ? sc.cut[k] : sc.cut_min;
+    // A group whose bound reaches this update's cut-off has its largest residual measured
+    // during the evaluation (warps with such a group run the tracking variant).
+    const bool may_shrink = k < a.iters && !(bound < cutk);
+    float e, sq, rmax;
+    if (__any_sync(wmask, may_shrink))
+      evaluate_any<E, WDT, true>(ws, w, s, z, step, qmax, pp, p_one, clamp, e, sq, rmax);
+    else
+      evaluate_any<E, WDT, false>(ws, w, s, z, step, qmax, pp, p_one, clamp, e, sq, rmax);
     if constexpr (L > 1) {
       e = group_sum<L>(e, gmask);
       sq = group_sum<L>(sq, gmask);
@@ -475,23 +516,25 @@ __device__ __forceinline__ void solve_group(const QArgs& a, int64_t g, int lane,
     }
     if (k == a.iters) break;
 
-    // Bound on max_j |r_j|: unclamped codes leave |v - Q| <= 1/2, clamped ones at most the
-    // distance of the group's extreme scaled weight from the code range.
-    const float hi = fmaxf(0.5f, fmaxf(-__fadd_rn(wsmin, z), __fsub_rn(__fadd_rn(wsmax, z), qmax)));
-    const float bound = step * (hi * 1.001f + 1e-3f * (fabsf(z) + qmax + 1.0f));
-    const bool no_shrink = bound < athr_lo;  // then also for every later update at this z
+    // The exact shrinkage runs only where a residual reaches the cut-off (then it also skips
+    // the elements below it); elsewhere every We is exactly 0.
+    bool shrink = false;
+    if (may_shrink) {
+      if constexpr (L > 1) rmax = group_max<L>(rmax, gmask);
+      shrink = !(rmax < cutk);
+    }
     // Closed-form zero. Every lane computes it (a masked warp instruction costs the pipe as
     // much as a full one, so one lane computing and broadcasting would only add a shuffle).
     float znew;
-    if (HQQ_F32_UPDATE && no_shrink && f32_update_exact) {
+    if (HQQ_F32_UPDATE && !shrink && f32_update_exact) {
       znew = __fmul_rn(__fsub_rn(sq, S_ws_f), 1.0f / (float)G);
     } else {
       // the definition's fp64 form z = fp32((sumQ - S_ws + s*sumWe) / G) (G = 2^k: the
-      // division is exact), with the exact shrinkage sum unless the bound rules it out
+      // division is exact), with the exact shrinkage sum where a residual reaches the cut-off
       double swe = 0.0;
-      if (!no_shrink) {
+      if (shrink) {
         swe = shrink_sum_exact<G, E, AXIS, WDT>(a, g, lane, s, step, z, __fdiv_rn(1.0f, beta),
-                                                athr_lo);
+                                                cutk);
         if constexpr (L > 1) swe = group_sum_d<L>(swe, gmask);
       }
       const double num = __dadd_rn(__dsub_rn(small_int_f32_to_f64(sq), (double)S_ws_f),
@@ -500,9 +543,10 @@ __device__ __forceinline__ void solve_group(const QArgs& a, int64_t g, int lane,
     }
     beta = __fmul_rn(beta, a.kappa);
     if constexpr (STOP) {
-      // Fixed point: same zero, provably no shrinkage from here on, so every remaining
-      // evaluation repeats this one exactly (same codes and error, never a new best).
-      const bool settled = no_shrink && __float_as_uint(znew) == __float_as_uint(z);
+      // Fixed point: same zero, and the bound is below every later update's cut-off, so
+      // every remaining evaluation repeats this one exactly (same codes and error, never a
+      // new best).
+      const bool settled = bound < sc.cut_min && __float_as_uint(znew) == __float_as_uint(z);
       z = znew;
       if (__all_sync(wmask, settled)) break;
     } else {
@@ -521,25 +565,13 @@ __device__ __forceinline__ void solve_group(const QArgs& a, int64_t g, int lane,
   zbest_out = zbest;
 }
 
-// Lower bound (absolute units) of the shrinkage cut-off |r| > beta_k^(-1/(2-p)) over all
-// updates: beta_k is non-decreasing, so the last update has the smallest cut-off. Lane 0 of
-// each warp computes it and broadcasts it (it only selects the exact path, never a result).
-__device__ __forceinline__ float shrink_cutoff_lower_bound(const QArgs& a) {
-  float athr = 0.0f;
-  if ((threadIdx.x & 31) == 0 && a.iters > 0) {
-    float b = a.beta0;
-    for (int k = 1; k < a.iters; ++k) b = __fmul_rn(b, a.kappa);
-    athr = powf(__fdiv_rn(1.0f, b), 1.0f / (2.0f - a.p)) * 0.998f;
-  }
-  return __shfl_sync(0xffffffffu, athr, 0);
-}
-
 // A batch of matrices sharing one configuration, passed by value as kernel parameters
 // (no device allocation): per-matrix pointers and shapes, and the prefix sums of their
 // tile counts, so that a block finds its matrix with a binary search in parameter space.
 template <int MAXB>
 struct QBatch {
   QArgs c;                         // shared settings; pointers/shape fields unused
+  ShrinkCut sc;                    // cut-offs of the updates (host-computed)
   int n;                           // matrices in this launch
   int64_t tile_start[MAXB + 1];    // tile_start[i] = first tile of matrix i
   const void* W[MAXB];
@@ -593,7 +625,6 @@ __global__ void __launch_bounds__(kQBlock, min_blocks<G, L>())
   const bool valid = g < a.n_groups;
   const unsigned wmask = __ballot_sync(0xffffffffu, valid);  // live lanes of this warp
   const unsigned gmask = L == 1 ? 0u : (((1u << L) - 1u) << ((tid & 31) & ~(L - 1)));
-  const float athr_lo = shrink_cutoff_lower_bound(a);
 
   // axis 0: the tile paths when every 16-byte piece stays in one row block (block-uniform)
   const bool tiled = (kTile || kWTile) && a.cols % elems_per_16B<WDT>() == 0;
@@ -618,7 +649,7 @@ __global__ void __launch_bounds__(kQBlock, min_blocks<G, L>())
     }
     uint32_t q[E];
     float step, zbest;
-    solve_group<G, L, AXIS, WDT, STOP>(a, g, lane, gmask, wmask, athr_lo, w, q, step, zbest);
+    solve_group<G, L, AXIS, WDT, STOP>(a, g, lane, gmask, wmask, batch.sc, w, q, step, zbest);
     if (lane == 0) {
       store_meta(a.scale, a.scale_dtype, g, step);
       store_meta(a.zero, a.zero_dtype, g, zbest);
@@ -662,6 +693,25 @@ __global__ void __launch_bounds__(kQBlock, min_blocks<G, L>())
 #define HQQ_G64_LANES 2
 #endif
 
+// Host side of ShrinkCut: beta_k and 1/beta_k by the kernel's fp32 operations (IEEE single
+// precision, round to nearest, on the host too), the power in fp64, rounded down to fp32.
+static void fill_cutoffs(int iters, float p, float beta0, float kappa, ShrinkCut* sc) {
+  const double e = 1.0 / (2.0 - (double)p);
+  float beta = beta0;
+  float last = 0.0f;
+  for (int k = 0; k < iters; ++k) {
+    const float ib = 1.0f / beta;
+    const double c = pow((double)ib, e) * (1.0 - 1e-5);
+    float cf = (float)c;
+    if ((double)cf > c) cf = nextafterf(cf, 0.0f);
+    if (k < kCutTable) sc->cut[k] = cf;
+    last = cf;
+    beta = beta * kappa;
+  }
+  for (int k = iters < kCutTable ? iters : kCutTable; k < kCutTable; ++k) sc->cut[k] = last;
+  sc->cut_min = last;
+}
+
 template <int MAXB>
 static cudaError_t fill_batch(const QuantJob* jobs, int n, int ngb, QBatch<MAXB>* b,
                               int64_t* tiles_out) {
@@ -680,6 +730,7 @@ static cudaError_t fill_batch(const QuantJob* jobs, int n, int ngb, QBatch<MAXB>
   c.scale_dtype = j0.scale_dtype;
   c.zero_dtype = j0.zero_dtype;
   c.flags = j0.flags;
+  fill_cutoffs(j0.iters, j0.p, j0.beta0, j0.kappa, &b->sc);
   int64_t tiles = 0;
   int k = 0;
   for (int i = 0; i < n; ++i) {
