@@ -872,6 +872,36 @@ SINGLE_CASES = {
 }
 
 
+def single_dequantize_block(reps: int = 10):
+    """The batched dequantize launch of the bench step on one Llama-7B block (7 matrices,
+    202M weights: 101 MB of codes and 6 MB of meta in, 405 MB of bf16 out): one launch, timed
+    over `reps` launches after warm-up (the ncu case of the batched dequantizer)."""
+    import calibration_free_weight_hqq_b200 as hqq
+    from calibration_free_weight_hqq_b200 import workloads
+    wl = workloads.llama7b_block_4b()
+    Ws = [workloads.make_weight(m, "cuda") for m in wl.matrices]
+    params = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16)
+    outs = hqq.hqq_quantize_batched(Ws, params)
+    shapes = [tuple(W.shape) for W in Ws]
+    D = [torch.empty_like(W) for W in Ws]
+    del Ws
+    b = hqq.matrix_batch(D, outs)
+    run = lambda: hqq.hqq_dequantize_batched(outs, shapes, params, W_out=D, batch=b)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    gbs = 2.5625 * wl.weights / (ms * 1e-3) / 1e9
+    return {"single": "dequantize_block_batched", "weights": wl.weights, "ms": round(ms, 4),
+            "GB_per_s_algorithmic": round(gbs, 1), "hbm_frac": round(gbs / peaks()["hbm_gbs"], 4)}
+
+
 def single(kind: str, reps: int = 10):
     """One matrix of SINGLE_CASES[kind]: time `reps` solver or dequantize launches after
     warm-up (the cases the ncu captures in profiles/ use)."""
@@ -924,7 +954,8 @@ def main():
                     help="leave the four smaller configurations out of the JSON line")
     ap.add_argument("--mixed", action="store_true",
                     help="whole model with per-layer configurations (8/4/2 bits) and exit")
-    ap.add_argument("--single", choices=sorted(SINGLE_CASES) + ["linear", "decode"],
+    ap.add_argument("--single", choices=sorted(SINGLE_CASES) + ["dequantize_block_batched",
+                                                                 "linear", "decode"],
                     help="time one matrix of a profiling case (SINGLE_CASES), one 4096^3 "
                          "linear layer, or one 4096x4096 layer at 16 tokens, and exit")
     args = ap.parse_args()
@@ -938,6 +969,8 @@ def main():
     if args.single:
         if args.single in ("linear", "decode"):
             print(json.dumps(single_linear(M=4096 if args.single == "linear" else 16)), flush=True)
+        elif args.single == "dequantize_block_batched":
+            print(json.dumps(single_dequantize_block()), flush=True)
         else:
             print(json.dumps(single(args.single)), flush=True)
         return

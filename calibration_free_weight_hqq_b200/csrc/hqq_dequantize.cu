@@ -79,6 +79,63 @@ __device__ __forceinline__ DArgs batch_args(const DBatch<MAXB>& b, int64_t tile,
   return a;
 }
 
+// The tiles of a persistent block: a contiguous range of ceil(total / gridDim.x) tiles, so
+// that the block finds its first matrix with one binary search and then only steps to the
+// next matrix when its range crosses a matrix boundary (a search per tile cost as many
+// instructions as the conversion of the tile's 32 elements per thread).
+template <int MAXB>
+struct TileCursor {
+  const DBatch<MAXB>& b;
+  int64_t t, t_end;   // next tile, end of the block's range
+  int64_t mstart;     // first tile of the current matrix
+  int64_t mend;       // first tile past the current matrix
+  int mi;             // current matrix
+  DArgs a;            // its arguments
+
+  __device__ explicit TileCursor(const DBatch<MAXB>& batch) : b(batch) {
+    const int64_t total = b.tile_start[b.n];
+    const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+    t = (int64_t)blockIdx.x * per;
+    t_end = t + per < total ? t + per : total;
+    mi = -1;
+    mstart = mend = 0;
+    if (t < t_end) {
+      int lo = 0, hi = b.n - 1;  // the last i with tile_start[i] <= t
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (b.tile_start[mid] <= t) lo = mid; else hi = mid - 1;
+      }
+      set(lo);
+    }
+  }
+  __device__ void set(int i) {
+    mi = i;
+    mstart = b.tile_start[i];
+    mend = b.tile_start[i + 1];
+    a = b.c;
+    a.packed = b.packed[i];
+    a.scale = b.scale[i];
+    a.zero = b.zero[i];
+    a.scale_mm = b.scale_mm[i];
+    a.zero_mm = b.zero_mm[i];
+    a.rows = b.rows[i];
+    a.cols = b.cols[i];
+    a.n = a.rows * a.cols;
+    a.out = b.out[i];
+  }
+  // Moves to the next tile of the range; false when the range is done. *local = the tile's
+  // index within its matrix.
+  __device__ bool next(int64_t* local) {
+    if (t >= t_end) return false;
+    int i = mi;
+    while (t >= mend) mend = b.tile_start[++i + 1];  // empty matrices have no tiles
+    if (i != mi) set(i);
+    *local = t - mstart;
+    ++t;
+    return true;
+  }
+};
+
 // Small non-negative integer (< 2^23) to fp32 without a conversion instruction: OR it into
 // the mantissa of 2^23 and subtract 2^23 (exact; stays on the FMA/ALU pipes).
 __device__ __forceinline__ float u2f_small(uint32_t q) {
@@ -182,12 +239,12 @@ __device__ __forceinline__ float code_magic(uint64_t field, int j) {
 template <int NB, int OUT_DT, int MAXB>
 __global__ void __launch_bounds__(kDBlock) dequant_axis1_kernel(
     const __grid_constant__ DBatch<MAXB> batch) {
-  const int64_t total = batch.tile_start[batch.n];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float2 neg_magic = make_float2(-8388608.0f, -8388608.0f);
-  for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
-    int64_t local;
-    const DArgs a = batch_args(batch, t, &local);
+  TileCursor<MAXB> cur(batch);
+  int64_t local;
+  while (cur.next(&local)) {
+    const DArgs& a = cur.a;
     const int64_t e0 = local * kDTile1;  // the tile's first element
     const int64_t left = a.n - e0;
     const int rem = left < kDTile1 ? (int)left : kDTile1;
@@ -242,11 +299,11 @@ constexpr int64_t kDTile4 = (int64_t)kDBlock * 8 * kD4Unroll;
 template <int OUT_DT, int MAXB>
 __global__ void __launch_bounds__(kDBlock) dequant4_axis1_kernel(
     const __grid_constant__ DBatch<MAXB> batch) {
-  const int64_t total = batch.tile_start[batch.n];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
-    int64_t local;
-    const DArgs a = batch_args(batch, t, &local);
+  TileCursor<MAXB> cur(batch);
+  int64_t local;
+  while (cur.next(&local)) {
+    const DArgs& a = cur.a;
     const int64_t base = local * kDTile4 + (int64_t)warp * (kD4Unroll * 256) + lane * 8;
     uint32_t w[kD4Unroll];
     float sc[kD4Unroll], zr[kD4Unroll];
@@ -326,11 +383,11 @@ __global__ void __launch_bounds__(kDBlock) dequant_axis0_cols_kernel(
   constexpr int kBg = G * NB / 8;  // bytes per group: 1, 2, 4 or 8
   constexpr int kWords = 2 * kBg;  // 8 groups
   static_assert(kBg == 1 || kBg == 2 || kBg == 4 || kBg == 8, "group bytes");
-  const int64_t total = batch.tile_start[batch.n];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
-    int64_t local;
-    const DArgs a = batch_args(batch, t, &local);
+  TileCursor<MAXB> cur(batch);
+  int64_t local;
+  while (cur.next(&local)) {
+    const DArgs& a = cur.a;
     const int64_t cunits = (a.cols + kD0Cols - 1) / kD0Cols;
     const int64_t unit = local * (kDBlock / 32) + warp;
     const int64_t rb = unit / cunits;
