@@ -473,7 +473,16 @@ def run_linear(hqq, dev, args, tokens: int = 4096):
         Yd = torch.empty(dec_tokens, m.rows, dtype=torch.bfloat16, device=dev)
         dec.append((m, Xd, pk, sc, zr, Yd, Wd))
 
+    # the weights were quantized and synchronised before: the decode launches may overlap the
+    # previous layer's tail (HQQ_FLAG_OVERLAP_WEIGHTS, programmatic dependent launch)
+    p_ovl = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16, meta_dtype=torch.bfloat16,
+                            overlap_weights=True)
+
     def dec_fused():
+        for m, Xd, pk, sc, zr, Yd, Wd in dec:
+            hqq.hqq_linear(Xd, pk, sc, zr, m.rows, p_ovl, Y=Yd)
+
+    def dec_fused_plain():
         for m, Xd, pk, sc, zr, Yd, Wd in dec:
             hqq.hqq_linear(Xd, pk, sc, zr, m.rows, Y=Yd)
 
@@ -482,6 +491,7 @@ def run_linear(hqq, dev, args, tokens: int = 4096):
             torch.matmul(Xd, Wd.t(), out=Yd)
 
     ms_dec = time_graph(capture_graph(dec_fused), args.warmup, args.steps, flush)
+    ms_dec_plain = time_graph(capture_graph(dec_fused_plain), args.warmup, args.steps, flush)
     ms_dec_cublas = time_graph(capture_graph(dec_cublas), args.warmup, args.steps, flush)
     dec_fused()  # leave the fused result in Yd
     wbytes = sum(m.rows * m.cols * (0.5 + 4 / 64) for m, *_ in dec)
@@ -506,6 +516,9 @@ def run_linear(hqq, dev, args, tokens: int = 4096):
                       "of up to 8 CTAs)",
             "timing": "CUDA graph of the 7 launches, L2 flushed before each replay",
             "ms_per_step": round(ms_dec, 4), "launches_per_step": len(dec),
+            "overlap": "HQQ_FLAG_OVERLAP_WEIGHTS (programmatic dependent launch: a layer's "
+                       "weight codes load while the previous layer finishes)",
+            "ms_per_step_without_overlap": round(ms_dec_plain, 4),
             "cublas_bf16_weight_ms_per_step": round(ms_dec_cublas, 4),
             "tflops": round(sum(2.0 * dec_tokens * m.rows * m.cols for m, *_ in dec)
                             / (ms_dec * 1e-3) / 1e12, 2),
@@ -706,9 +719,10 @@ def run_reference(args, rank, world):
 
 def single_linear(reps: int = 10, M: int = 4096):
     """One 4096 x 4096 hqq_linear launch with M tokens (bf16, 4-bit g64): the ncu profiling
-    cases (M = 4096: the 2-SM kernel; M = 16: the decode kernel). `reps` launches are
-    captured in one CUDA graph (a decode launch is shorter than the binding's host time) and
-    the replay is timed; the weight (8.4 MB of codes) stays in L2 between launches."""
+    cases (M = 4096: the 2-SM kernel; M = 16: the decode kernel, launched with
+    HQQ_FLAG_OVERLAP_WEIGHTS). `reps` launches are captured in one CUDA graph (a decode launch
+    is shorter than the binding's host time) and the replay is timed; the weight (8.4 MB of
+    codes) stays in L2 between launches."""
     import calibration_free_weight_hqq_b200 as hqq
     from calibration_free_weight_hqq_b200 import synthetic
     N = K = 4096
@@ -717,9 +731,11 @@ def single_linear(reps: int = 10, M: int = 4096):
     X = synthetic.activations(M, K, seed=12, device="cuda")
     Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
 
+    p = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16, overlap_weights=True)
+
     def launches():
         for _ in range(reps):
-            hqq.hqq_linear(X, pk, s, z, N, Y=Y)
+            hqq.hqq_linear(X, pk, s, z, N, p, Y=Y)
 
     graph = capture_graph(launches)
     graph.replay()

@@ -66,6 +66,7 @@ class HQQParams(ctypes.Structure):
                 ("flags", ctypes.c_int)]
 
 HQQ_FLAG_STOP_AT_FIXED_POINT = 1
+HQQ_FLAG_OVERLAP_WEIGHTS = 2
 
 
 def library_path() -> str:
@@ -184,12 +185,16 @@ def _meta_shape(rows: int, cols: int, group_size: int, axis: int):
 
 def make_params(nbits=4, group_size=64, axis=1, iters=20, p=0.7, beta0=10.0, kappa=1.01,
                 w_dtype=torch.bfloat16, meta_dtype=None, quant_scale=False, quant_zero=False,
-                meta_group_size=128, stop_at_fixed_point=False) -> HQQParams:
+                meta_group_size=128, stop_at_fixed_point=False,
+                overlap_weights=False) -> HQQParams:
+    """The C struct hqq_params. stop_at_fixed_point: HQQ_FLAG_STOP_AT_FIXED_POINT (quantize);
+    overlap_weights: HQQ_FLAG_OVERLAP_WEIGHTS (hqq_linear; see the header for its promise)."""
     meta_dtype = w_dtype if meta_dtype is None else meta_dtype
+    flags = (HQQ_FLAG_STOP_AT_FIXED_POINT if stop_at_fixed_point else 0) | \
+        (HQQ_FLAG_OVERLAP_WEIGHTS if overlap_weights else 0)
     return HQQParams(nbits, group_size, axis, iters, p, beta0, kappa, _TORCH_DT[w_dtype],
                      _TORCH_DT[meta_dtype], int(bool(quant_scale)), int(bool(quant_zero)),
-                     meta_group_size,
-                     HQQ_FLAG_STOP_AT_FIXED_POINT if stop_at_fixed_point else 0)
+                     meta_group_size, flags)
 
 
 def hqq_workspace_bytes(rows: int, cols: int, params: HQQParams) -> int:

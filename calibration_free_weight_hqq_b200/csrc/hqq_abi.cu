@@ -528,6 +528,8 @@ HQQ_EXPORT hqq_status hqq_linear(const void* X, int64_t M, int64_t K, hqq_dtype 
       prm.quant_zero)
     return HQQ_ERR_UNSUPPORTED;
   if (!wdtype_ok(prm.meta_dtype)) return HQQ_ERR_INVALID_ARG;
+  if ((prm.flags & ~(HQQ_FLAG_STOP_AT_FIXED_POINT | HQQ_FLAG_OVERLAP_WEIGHTS)) != 0)
+    return HQQ_ERR_INVALID_ARG;
   if (K % 64 != 0 || N % 8 != 0) return HQQ_ERR_SHAPE;
   if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) ||
       (N + 255) / 256 > 65535)
@@ -554,6 +556,7 @@ HQQ_EXPORT hqq_status hqq_linear(const void* X, int64_t M, int64_t K, hqq_dtype 
   j.K = K;
   j.x_dtype = x_dtype;
   j.meta_dtype = prm.meta_dtype;
+  j.overlap_weights = (prm.flags & HQQ_FLAG_OVERLAP_WEIGHTS) != 0;
   return cuda_status(hqqk::launch_w4a16_gemm(j, stream));
 }
 

@@ -962,6 +962,7 @@ __global__ void __launch_bounds__(skinny::kThreads, 2)
 #ifndef HQQ_GEMV_DEPTH
 #define HQQ_GEMV_DEPTH 4
 #endif
+
 namespace gemv {
 constexpr int kWarps = HQQ_GEMV_WARPS;
 constexpr int kThreads = 32 * kWarps;
@@ -1054,9 +1055,15 @@ __global__ void __launch_bounds__(gemv::kThreads) w4a16_gemv_kernel(
       }
     }
   };
+  // Programmatic dependent launch (HQQ_FLAG_OVERLAP_WEIGHTS): the next kernel on the stream
+  // may start now; this one loads its weight codes and meta (which no earlier work writes, by
+  // the flag's promise) and then waits for the previous kernel's completion and memory before
+  // it reads X or writes anything. Without the launch attribute both are no-ops.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < kDepth; ++i)
     if (i < nloc) load_kb(i, code[i], msc[i], mzr[i]);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // X[0..15][slice] -> shared memory: 16-byte piece q (k = 8q within the slice) of token m at
   // m * rs + (q / 16) * 256 + (q % 4) * 64 + ((q / 4) % 4) * 16; zeros past M and past K
@@ -1203,10 +1210,12 @@ cudaError_t launch_typed(const GemmJob& job, cudaStream_t stream) {
   a.K = static_cast<int>(job.K);
   cudaLaunchConfig_t cfg = {};
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   CUtensorMap mx, mw;
@@ -1225,6 +1234,7 @@ cudaError_t launch_typed(const GemmJob& job, cudaStream_t stream) {
     cfg.blockDim = dim3(gemv::kThreads);
     cfg.dynamicSmemBytes = smem;
     attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    if (job.overlap_weights) cfg.numAttrs = 2;  // the decode kernel waits before reading X
     const uint8_t* packed = job.packed;
     const int lg_s = S == 8 ? 3 : S == 4 ? 2 : S == 2 ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, w4a16_gemv_kernel<F16, MT>, job.X, packed, a, lg_s, kb_per);

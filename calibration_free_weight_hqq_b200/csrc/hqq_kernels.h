@@ -62,6 +62,8 @@ struct GemmJob {
   int64_t M, N, K;
   int x_dtype;
   int meta_dtype;
+  bool overlap_weights;  // HQQ_FLAG_OVERLAP_WEIGHTS: the decode kernel may overlap the
+                         // previous kernel on the stream (programmatic dependent launch)
 };
 cudaError_t launch_w4a16_gemm(const GemmJob& job, cudaStream_t stream);
 // Number of bounded waits inside the GEMM kernel that ran out of time since the library was

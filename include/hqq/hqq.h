@@ -112,6 +112,17 @@ typedef struct {
  * evaluations per group. */
 #define HQQ_FLAG_STOP_AT_FIXED_POINT 1
 
+/* hqq_linear only (the quantize entry points refuse it): the caller promises that no work
+ * enqueued earlier on the stream, and possibly still running, writes this call's weight
+ * (Wq_packed, scale, zero) - as in a sequence of decode steps over weights quantized and
+ * synchronised beforehand. The decode kernel (M <= 16) may then start while the previous
+ * kernel on the stream is finishing (programmatic dependent launch): it loads its weight codes
+ * and meta first and waits for the previous kernel to complete, with its writes visible,
+ * before it reads X, bias or anything else and before it writes Y. Results are identical with
+ * or without the flag; other kernels ignore it. Without the promise (say, a quantize call just
+ * before on the same stream), leave it off. */
+#define HQQ_FLAG_OVERLAP_WEIGHTS 2
+
 /* Number of quantization groups of a [rows, cols] weight: rows*cols/group_size.
  * Returns -1 if the grouped dimension (cols for axis=1, rows for axis=0) is not a multiple
  * of group_size or an argument is out of range. Host only; no CUDA call. */
@@ -311,7 +322,9 @@ hqq_status hqq_dequantize_meta(const void* q_u8, const void* mm, int64_t n, int 
  * Shapes: K % 64 == 0 and N % 8 == 0 (HQQ_ERR_SHAPE otherwise), M, K < 2^31, N <= 65535*256.
  * K == 0 gives
  * Y = bias (or 0). Other nbits / group_size / axis, or quant_scale / quant_zero, return
- * HQQ_ERR_UNSUPPORTED. The solver fields of params are ignored. */
+ * HQQ_ERR_UNSUPPORTED. The solver fields of params are ignored; params->flags may hold
+ * HQQ_FLAG_OVERLAP_WEIGHTS (and HQQ_FLAG_STOP_AT_FIXED_POINT, ignored), other bits return
+ * HQQ_ERR_INVALID_ARG. */
 hqq_status hqq_linear(const void* X, int64_t M, int64_t K, hqq_dtype x_dtype,
                       const void* Wq_packed, const void* scale, const void* zero,
                       const void* bias, int64_t N, const hqq_params* params, void* Y,

@@ -220,6 +220,18 @@ def test_linear_validates_before_launch(L):
     bad_meta = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16)
     bad_meta.meta_dtype = 3
     assert call(prm=bad_meta) == INVALID
+    # flags: the overlap promise (and the solver's fixed-point flag, ignored) are accepted
+    # (the call then fails only for its fake pointers, after validation); other bits are not
+    bad_flags = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16)
+    bad_flags.flags = 4
+    assert call(prm=bad_flags) == INVALID
+    ok_flags = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16, overlap_weights=True,
+                               stop_at_fixed_point=True)
+    assert call(prm=ok_flags, K=96) == SHAPE  # validation continues past the flags
+    # the quantize entry points refuse the linear layer's flag
+    ovl = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16, overlap_weights=True)
+    assert L.hqq_quantize_ex(FAKE, 64, 128, ctypes.byref(ovl), FAKE, FAKE, FAKE, None, None,
+                             None, 0, None) == INVALID
     assert call(K=96) == SHAPE
     assert call(N=260) == SHAPE
     assert call(M=1 << 31) == SHAPE

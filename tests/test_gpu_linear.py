@@ -268,3 +268,47 @@ def test_linear_decode_is_deterministic():
     a = run_linear(X, dev16, N, "f16", "f16")
     b = run_linear(X, dev16, N, "f16", "f16")
     assert np.array_equal(a, b)
+
+
+def test_linear_decode_overlap_flag_keeps_every_dependency():
+    """HQQ_FLAG_OVERLAP_WEIGHTS lets a decode launch start while the previous kernel on the
+    stream finishes; it must still read X only after that kernel is done. A chain of decode
+    layers where layer i+1 reads layer i's output, launched back to back on one stream with
+    nothing in between, must give bit for bit what the same chain gives without the flag (a
+    layer that read its X early would see the stale buffer, which holds other values), and
+    one-hot rows through flagged launches must still return the dequantized weight."""
+    N = K = 1024
+    M = 16
+    layers = [make_layer(N, K, 900 + i)[3] for i in range(6)]
+    X0 = make_x(M, K, 77, "bf16").cuda()
+
+    def chain(flag):
+        p = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16, meta_dtype=torch.bfloat16,
+                            overlap_weights=flag)
+        bufs = [torch.full((M, N), 3.0, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        x = X0
+        for i, dev in enumerate(layers):
+            y = bufs[i % 2]
+            hqq.hqq_linear(x, dev["packed"], dev["scale"], dev["zero"], N, p, Y=y)
+            x = y
+        torch.cuda.synchronize()
+        return x.float().cpu().numpy()
+
+    plain, overlapped = chain(False), chain(True)
+    assert np.isfinite(plain).all()
+    assert np.array_equal(plain, overlapped)
+    # one-hot through a flagged launch right after another flagged launch
+    codes, scale, zero, dev = make_layer(264, 2112, 32)
+    ks = 131 * np.arange(M) + 7
+    X = torch.zeros(M, 2112, dtype=torch.bfloat16)
+    X[torch.arange(M), torch.from_numpy(ks)] = 1.0
+    p = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16, meta_dtype=torch.bfloat16,
+                        overlap_weights=True)
+    Xc = X.cuda()
+    Y1 = hqq.hqq_linear(Xc, dev["packed"], dev["scale"], dev["zero"], 264, p)
+    Y2 = hqq.hqq_linear(Xc, dev["packed"], dev["scale"], dev["zero"], 264, p)
+    torch.cuda.synchronize()
+    Wd = oracle.round_to_dtype(oracle.dequantize(codes, scale, zero, 264, 2112, 64, 1), "bf16")
+    for Y in (Y1, Y2):
+        assert np.array_equal(Y.float().cpu().numpy(), Wd[:, ks].T)
+    assert_no_timeouts()
