@@ -11,7 +11,14 @@
 
 namespace hqqk {
 
-constexpr int kQBlock = 160;  // 5 warps; kQBlock*E codes per block is a multiple of 10
+// Threads per block: 160 (5 warps) for 3-bit codes, where 160*E codes per block must be a
+// multiple of 10 so that 10-code words never straddle blocks; HQQ_QBLOCK (4 warps by default)
+// otherwise, which with 128 registers a thread lets 16 warps share an SM instead of 15.
+#ifndef HQQ_QBLOCK
+#define HQQ_QBLOCK 128
+#endif
+template <bool PACK3>
+__host__ __device__ constexpr int qblock() { return PACK3 ? 160 : HQQ_QBLOCK; }
 
 // Tuning knobs (compile-time): minimum resident blocks per SM (0: the per-shape table
 // min_blocks below; a positive value forces it for every shape), and whether to round with
@@ -46,11 +53,12 @@ constexpr int kQBlock = 160;  // 5 warps; kQBlock*E codes per block is a multipl
 
 // Resident blocks per SM the register budget is sized for (measured on B200, every shape of
 // the shipped workloads): with 32 elements per lane the raw and scaled weights take 48
-// registers, and 3 blocks (128 registers a thread, no spills) ran faster than 4 or 5 (96 or
-// 72 registers, spills); with 16 or fewer elements per lane 4 blocks fit without spills.
-template <int G, int L>
+// registers, and 128 registers a thread (no spills) ran faster than 96 or 72 (spills); with
+// 16 or fewer elements per lane 96 registers fit without spills.
+template <int G, int L, int BLOCK>
 __host__ __device__ constexpr int min_blocks() {
-  return HQQ_MINB > 0 ? HQQ_MINB : (G / L < 32 ? 4 : 3);
+  // 32-element lanes: 128 registers (15 or 16 warps an SM); fewer elements: 96 (20 warps)
+  return HQQ_MINB > 0 ? HQQ_MINB : (G / L < 32 ? 640 : 512) / BLOCK;
 }
 
 __device__ __forceinline__ float round_even(float v) {
@@ -184,14 +192,14 @@ __device__ __forceinline__ void load_group(const QArgs& a, int64_t g, int lane, 
 template <int WDT>
 __host__ __device__ constexpr int elems_per_16B() { return WDT == kF32 ? 4 : 8; }
 
-template <int G, int NGB, int WDT>
+template <int G, int NGB, int WDT, int BLOCK>
 __device__ __forceinline__ void load_tile_axis0(const QArgs& a, int64_t g0, unsigned char* s_tile) {
   constexpr int PERV = elems_per_16B<WDT>();
   constexpr int ESZ = WDT == kF32 ? 4 : 2;
   constexpr int CPR = NGB / PERV;  // 16-byte pieces per element row of the tile
   const char* W = reinterpret_cast<const char*>(a.W);
 #pragma unroll 1
-  for (int k = threadIdx.x; k < G * CPR; k += kQBlock) {
+  for (int k = threadIdx.x; k < G * CPR; k += BLOCK) {
     const int j = k / CPR, i0 = (k - j * CPR) * PERV;
     const int64_t gg = g0 + i0;
     if (gg < a.n_groups) {
@@ -596,8 +604,9 @@ __device__ __forceinline__ int find_matrix(const QBatch<MAXB>& b, int64_t tile) 
 // each block's load / min-max / packing phases (a persistent grid-stride variant, where all
 // warps of an SM reach those phases together, measured 28 % slower).
 template <int G, int L, int AXIS, int WDT, bool PACK3, int MAXB, bool STOP>
-__global__ void __launch_bounds__(kQBlock, min_blocks<G, L>())
+__global__ void __launch_bounds__(qblock<PACK3>(), min_blocks<G, L, qblock<PACK3>()>())
     quantize_kernel(const __grid_constant__ QBatch<MAXB> batch) {
+  constexpr int kQBlock = qblock<PACK3>();
   constexpr int E = G / L;
   constexpr int NGB = kQBlock / L;  // groups per block
   __shared__ uint8_t s_codes[PACK3 ? NGB * G : 1];
@@ -632,7 +641,7 @@ __global__ void __launch_bounds__(kQBlock, min_blocks<G, L>())
   unsigned char* s_w = s_tile + (tid / 32) * (kWTile ? kWRegion : 0);
   if (tiled) {
     if constexpr (kTile) {
-      load_tile_axis0<G, NGB, WDT>(a, tile * NGB, s_tile);
+      load_tile_axis0<G, NGB, WDT, kQBlock>(a, tile * NGB, s_tile);
       __syncthreads();
     } else if constexpr (kWTile) {
       load_warp_tile_axis0<G, L, WDT>(a, tile * NGB + (tid / 32) * (32 / L), tid & 31, s_w);
@@ -754,16 +763,17 @@ static cudaError_t fill_batch(const QuantJob* jobs, int n, int ngb, QBatch<MAXB>
 
 template <int G, int L, int AXIS, int WDT, int MAXB, bool STOP>
 static cudaError_t launch_g(const QuantJob* jobs, int n, cudaStream_t st) {
-  constexpr int NGB = kQBlock / L;
+  const bool pack3 = jobs[0].nbits == 3;
+  const int block = pack3 ? qblock<true>() : qblock<false>();
   QBatch<MAXB> b;
   int64_t tiles = 0;
-  cudaError_t e = fill_batch<MAXB>(jobs, n, NGB, &b, &tiles);
+  cudaError_t e = fill_batch<MAXB>(jobs, n, block / L, &b, &tiles);
   if (e != cudaSuccess) return e;
   if (tiles == 0) return cudaSuccess;
-  if (jobs[0].nbits == 3) {
-    quantize_kernel<G, L, AXIS, WDT, true, MAXB, STOP><<<(unsigned)tiles, kQBlock, 0, st>>>(b);
+  if (pack3) {
+    quantize_kernel<G, L, AXIS, WDT, true, MAXB, STOP><<<(unsigned)tiles, block, 0, st>>>(b);
   } else {
-    quantize_kernel<G, L, AXIS, WDT, false, MAXB, STOP><<<(unsigned)tiles, kQBlock, 0, st>>>(b);
+    quantize_kernel<G, L, AXIS, WDT, false, MAXB, STOP><<<(unsigned)tiles, block, 0, st>>>(b);
   }
   return cudaGetLastError();
 }
