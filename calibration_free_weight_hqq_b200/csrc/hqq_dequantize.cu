@@ -79,59 +79,77 @@ __device__ __forceinline__ DArgs batch_args(const DBatch<MAXB>& b, int64_t tile,
   return a;
 }
 
-// The tiles of a persistent block: a contiguous range of ceil(total / gridDim.x) tiles, so
-// that the block finds its first matrix with one binary search and then only steps to the
-// next matrix when its range crosses a matrix boundary (a search per tile cost as many
-// instructions as the conversion of the tile's 32 elements per thread).
+// The tiles of a persistent block. HQQ_DQ_ORDER 0: grid-stride order (tiles b, b + grid, ...),
+// so that the resident blocks work on one contiguous band of the output at a time; 1: a
+// contiguous range of ceil(total / grid) tiles per block. Either way a block's tile index only
+// grows, so it finds its first matrix with one binary search and afterwards only steps forward
+// over matrix boundaries (a search per tile cost as many instructions as the conversion of the
+// tile's 32 elements per thread).
+#ifndef HQQ_DQ_ORDER
+#define HQQ_DQ_ORDER 0
+#endif
+template <int MAXB>
+__device__ __forceinline__ DArgs matrix_args(const DBatch<MAXB>& b, int i) {
+  DArgs a = b.c;
+  a.packed = b.packed[i];
+  a.scale = b.scale[i];
+  a.zero = b.zero[i];
+  a.scale_mm = b.scale_mm[i];
+  a.zero_mm = b.zero_mm[i];
+  a.rows = b.rows[i];
+  a.cols = b.cols[i];
+  a.n = a.rows * a.cols;
+  a.out = b.out[i];
+  return a;
+}
+
+// The cursor holds only the matrix index and its tile range; a tile's arguments are read from
+// the parameter space when the tile starts (holding them across tiles cost up to 23 registers
+// and occupancy in these memory-bound kernels).
 template <int MAXB>
 struct TileCursor {
   const DBatch<MAXB>& b;
-  int64_t t, t_end;   // next tile, end of the block's range
-  int64_t mstart;     // first tile of the current matrix
-  int64_t mend;       // first tile past the current matrix
-  int mi;             // current matrix
-  DArgs a;            // its arguments
+  int64_t t, t_end, stride;  // next tile, end, step between a block's tiles
+  int64_t mstart;            // first tile of the current matrix
+  int64_t mend;              // first tile past the current matrix
+  int mi;                    // current matrix
 
   __device__ explicit TileCursor(const DBatch<MAXB>& batch) : b(batch) {
     const int64_t total = b.tile_start[b.n];
-    const int64_t per = (total + gridDim.x - 1) / gridDim.x;
-    t = (int64_t)blockIdx.x * per;
-    t_end = t + per < total ? t + per : total;
-    mi = -1;
-    mstart = mend = 0;
+    if (HQQ_DQ_ORDER == 0) {
+      t = blockIdx.x;
+      t_end = total;
+      stride = gridDim.x;
+    } else {
+      const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+      t = (int64_t)blockIdx.x * per;
+      t_end = t + per < total ? t + per : total;
+      stride = 1;
+    }
+    mi = 0;
     if (t < t_end) {
       int lo = 0, hi = b.n - 1;  // the last i with tile_start[i] <= t
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (b.tile_start[mid] <= t) lo = mid; else hi = mid - 1;
       }
-      set(lo);
+      mi = lo;
     }
+    mstart = b.tile_start[mi];
+    mend = b.tile_start[mi + 1];
   }
-  __device__ void set(int i) {
-    mi = i;
-    mstart = b.tile_start[i];
-    mend = b.tile_start[i + 1];
-    a = b.c;
-    a.packed = b.packed[i];
-    a.scale = b.scale[i];
-    a.zero = b.zero[i];
-    a.scale_mm = b.scale_mm[i];
-    a.zero_mm = b.zero_mm[i];
-    a.rows = b.rows[i];
-    a.cols = b.cols[i];
-    a.n = a.rows * a.cols;
-    a.out = b.out[i];
-  }
-  // Moves to the next tile of the range; false when the range is done. *local = the tile's
-  // index within its matrix.
-  __device__ bool next(int64_t* local) {
+  // Moves to the block's next tile; false when there is none. *local = the tile's index
+  // within its matrix, *matrix = the matrix.
+  __device__ bool next(int64_t* local, int* matrix) {
     if (t >= t_end) return false;
-    int i = mi;
-    while (t >= mend) mend = b.tile_start[++i + 1];  // empty matrices have no tiles
-    if (i != mi) set(i);
+    while (t >= mend) {  // empty matrices have no tiles
+      ++mi;
+      mstart = mend;
+      mend = b.tile_start[mi + 1];
+    }
     *local = t - mstart;
-    ++t;
+    *matrix = mi;
+    t += stride;
     return true;
   }
 };
@@ -243,8 +261,9 @@ __global__ void __launch_bounds__(kDBlock) dequant_axis1_kernel(
   const float2 neg_magic = make_float2(-8388608.0f, -8388608.0f);
   TileCursor<MAXB> cur(batch);
   int64_t local;
-  while (cur.next(&local)) {
-    const DArgs& a = cur.a;
+  int mi;
+  while (cur.next(&local, &mi)) {
+    const DArgs a = matrix_args(batch, mi);
     const int64_t e0 = local * kDTile1;  // the tile's first element
     const int64_t left = a.n - e0;
     const int rem = left < kDTile1 ? (int)left : kDTile1;
@@ -302,8 +321,9 @@ __global__ void __launch_bounds__(kDBlock) dequant4_axis1_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   TileCursor<MAXB> cur(batch);
   int64_t local;
-  while (cur.next(&local)) {
-    const DArgs& a = cur.a;
+  int mi;
+  while (cur.next(&local, &mi)) {
+    const DArgs a = matrix_args(batch, mi);
     const int64_t base = local * kDTile4 + (int64_t)warp * (kD4Unroll * 256) + lane * 8;
     uint32_t w[kD4Unroll];
     float sc[kD4Unroll], zr[kD4Unroll];
@@ -386,8 +406,9 @@ __global__ void __launch_bounds__(kDBlock) dequant_axis0_cols_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   TileCursor<MAXB> cur(batch);
   int64_t local;
-  while (cur.next(&local)) {
-    const DArgs& a = cur.a;
+  int mi;
+  while (cur.next(&local, &mi)) {
+    const DArgs a = matrix_args(batch, mi);
     const int64_t cunits = (a.cols + kD0Cols - 1) / kD0Cols;
     const int64_t unit = local * (kDBlock / 32) + warp;
     const int64_t rb = unit / cunits;
