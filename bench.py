@@ -755,62 +755,45 @@ def configs_table(reps: int = 5):
     """Quantize and dequantize throughput of the four smaller workloads of the pages'
     configurations (the fifth, the whole model, is the headline), one line per configuration:
     solver Gweights/s and its MUFU fraction, dequantizer algorithmic GB/s and its HBM fraction.
-    Quantize: each matrix timed with CUDA events over `reps` launches after one warm-up (a
-    launch takes milliseconds, so host gaps do not matter). Dequantize: one pass over all the
-    workload's matrices is captured in a CUDA graph (so that the microsecond launches run back
-    to back, without the binding's host time between them); L2 is flushed (256 MB write)
-    before each of `reps` timed replays, which are timed one by one and averaged."""
+
+    A workload whose matrices share one configuration without second-level meta (the Llama
+    block at 4-bit and at 2-bit axis 0) is quantized and dequantized with the batched calls, one
+    launch each, as a caller quantizing a block would; the others (one matrix; the 70B MLP with
+    two bit widths and 8-bit meta, through hqq_quantize_ex) take a call per matrix, and the
+    per-matrix figures are reported for every workload. Quantize: `reps` back-to-back calls
+    timed with CUDA events after one warm-up (a launch takes milliseconds, so host gaps do not
+    matter). Dequantize: one pass captured in a CUDA graph (so that microsecond launches run
+    back to back), L2 flushed (256 MB write) before each of `reps` timed replays."""
     import calibration_free_weight_hqq_b200 as hqq
     from calibration_free_weight_hqq_b200 import workloads
     pk = peaks()
     mufu_peak = MUFU_PER_CLK_PER_SM * N_SM * pk["sm_max_mhz"] * 1e6
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    out = []
-    for wl in (workloads.single_fp16(), workloads.llama7b_block_4b(),
-               workloads.llama7b_block_2b_axis0(), workloads.mlp70b_mixed()):
-        q_ms = 0.0
-        dq_bytes = 0
-        passes = []  # (q, rows, cols, params, dtype, D) per matrix
-        for m in wl.matrices:
-            W = workloads.make_weight(m, "cuda")
-            params = hqq.make_params(m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0,
-                                     m.kappa, w_dtype=m.dtype, quant_scale=m.quant_meta,
-                                     quant_zero=m.quant_meta,
-                                     meta_group_size=m.meta_group_size)
-            need = hqq.hqq_workspace_bytes(m.rows, m.cols, params)
-            ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda") if need else None
-            q = hqq.hqq_quantize_ex(W, params, workspace=ws)
-            hqq.hqq_quantize_ex(W, params, out=q, workspace=ws)
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(reps):
-                hqq.hqq_quantize_ex(W, params, out=q, workspace=ws)
-            e1.record()
-            torch.cuda.synchronize()
-            q_ms += e0.elapsed_time(e1) / reps
-            passes.append((q, m.rows, m.cols, params, m.dtype, torch.empty_like(W)))
-            ng = m.numel // m.group_size
-            meta_b = 2 * ng * (1 if m.quant_meta else 2)
-            dq_bytes += hqq.hqq_packed_bytes(m.rows, m.cols, m.nbits) + meta_b + 2 * m.numel
-            del W, ws
 
-        def dequantize_all():
-            for q, rows, cols, params, dt, D in passes:
-                hqq.hqq_dequantize_ex(q, rows, cols, params, out_dtype=dt, out=D)
+    def events_ms(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
 
-        dequantize_all()
+    def graph_ms(fn):
+        fn()
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
             with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
-                dequantize_all()
+                fn()
         torch.cuda.current_stream().wait_stream(side)
         graph.replay()
         torch.cuda.synchronize()
-        d_ms = 0.0
+        total = 0.0
         for _ in range(reps):
             flush.fill_(1)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -818,17 +801,71 @@ def configs_table(reps: int = 5):
             graph.replay()
             e1.record()
             torch.cuda.synchronize()
-            d_ms += e0.elapsed_time(e1) / reps
-        del graph, passes
+            total += e0.elapsed_time(e1) / reps
+        del graph
+        return total
+
+    out = []
+    for wl in (workloads.single_fp16(), workloads.llama7b_block_4b(),
+               workloads.llama7b_block_2b_axis0(), workloads.mlp70b_mixed()):
+        Ws = [workloads.make_weight(m, "cuda") for m in wl.matrices]
+        plist = [hqq.make_params(m.nbits, m.group_size, m.axis, m.iters, m.p, m.beta0, m.kappa,
+                                 w_dtype=m.dtype, quant_scale=m.quant_meta,
+                                 quant_zero=m.quant_meta, meta_group_size=m.meta_group_size)
+                 for m in wl.matrices]
+        dq_bytes = 0
+        for m in wl.matrices:
+            ng = m.numel // m.group_size
+            meta_b = 2 * ng * (1 if m.quant_meta else 2)
+            dq_bytes += hqq.hqq_packed_bytes(m.rows, m.cols, m.nbits) + meta_b + 2 * m.numel
+        # per matrix: hqq_quantize_ex / hqq_dequantize_ex
+        passes, q_ms_per = [], 0.0
+        for m, W, params in zip(wl.matrices, Ws, plist):
+            need = hqq.hqq_workspace_bytes(m.rows, m.cols, params)
+            ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda") if need else None
+            q = hqq.hqq_quantize_ex(W, params, workspace=ws)
+            q_ms_per += events_ms(lambda: hqq.hqq_quantize_ex(W, params, out=q, workspace=ws))
+            passes.append((q, m.rows, m.cols, params, m.dtype, torch.empty_like(W)))
+
+        def dequantize_all():
+            for q, rows, cols, params, dt, D in passes:
+                hqq.hqq_dequantize_ex(q, rows, cols, params, out_dtype=dt, out=D)
+        d_ms_per = graph_ms(dequantize_all)
         n = wl.weights
-        mufu = 2 * (wl.matrices[0].iters + 1) * n / (q_ms * 1e-3)
+        nit = 2 * (wl.matrices[0].iters + 1)
+        line = {"workload": wl.name, "weights": n}
+        batched = len(wl.matrices) > 1 and not any(m.quant_meta for m in wl.matrices) and \
+            all((m.nbits, m.group_size, m.axis, m.dtype) == (wl.matrices[0].nbits,
+                wl.matrices[0].group_size, wl.matrices[0].axis, wl.matrices[0].dtype)
+                for m in wl.matrices)
+        if batched:
+            p0 = plist[0]
+            outs = hqq.hqq_quantize_batched(Ws, p0)
+            qb = hqq.matrix_batch(Ws, outs)
+            q_ms = events_ms(lambda: hqq.hqq_quantize_batched(Ws, p0, outs=outs, batch=qb))
+            shapes = [tuple(W.shape) for W in Ws]
+            Ds = [torch.empty_like(W) for W in Ws]
+            db = hqq.matrix_batch(Ds, outs)
+            d_ms = graph_ms(lambda: hqq.hqq_dequantize_batched(outs, shapes, p0, W_out=Ds,
+                                                                batch=db))
+            line["calls"] = "hqq_quantize_batched + hqq_dequantize_batched (one launch each)"
+            del outs, Ds
+        else:
+            q_ms, d_ms = q_ms_per, d_ms_per
+            line["calls"] = "hqq_quantize_ex + hqq_dequantize_ex per matrix"
         gbs = dq_bytes / (d_ms * 1e-3) / 1e9
-        out.append({"workload": wl.name, "weights": n,
-                    "quantize_ms": round(q_ms, 3), "quantize_Gweights_per_s": round(n / q_ms / 1e6, 2),
-                    "quantize_mufu_frac": round(mufu / mufu_peak, 4),
-                    "dequantize_ms": round(d_ms, 4), "dequantize_GB_per_s": round(gbs, 1),
-                    "dequantize_hbm_frac": round(gbs / pk["hbm_gbs"], 4),
-                    "dequantize_timing": "CUDA graph of one pass, L2 flushed before each replay"})
+        gbs_per = dq_bytes / (d_ms_per * 1e-3) / 1e9
+        line.update({
+            "quantize_ms": round(q_ms, 3), "quantize_Gweights_per_s": round(n / q_ms / 1e6, 2),
+            "quantize_mufu_frac": round(nit * n / (q_ms * 1e-3) / mufu_peak, 4),
+            "dequantize_ms": round(d_ms, 4), "dequantize_GB_per_s": round(gbs, 1),
+            "dequantize_hbm_frac": round(gbs / pk["hbm_gbs"], 4),
+            "per_matrix_quantize_mufu_frac": round(nit * n / (q_ms_per * 1e-3) / mufu_peak, 4),
+            "per_matrix_dequantize_hbm_frac": round(gbs_per / pk["hbm_gbs"], 4),
+            "dequantize_timing": "CUDA graph of one pass, L2 flushed before each replay"})
+        out.append(line)
+        del passes, Ws
+        torch.cuda.empty_cache()
     return out
 
 
