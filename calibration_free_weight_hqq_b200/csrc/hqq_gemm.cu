@@ -977,7 +977,7 @@ constexpr int kMaxM = 16;
 constexpr uint32_t kRedBytes = kRowsCta * 16 * 4;
 __host__ __device__ constexpr uint32_t x_row_bytes(int kb_per) { return kb_per * 256 + 64; }
 __host__ __device__ constexpr uint32_t smem_bytes(int kb_per) {
-  return 16 * x_row_bytes(kb_per) + kRedBytes;
+  return 16 * x_row_bytes(kb_per) + 2 * kRedBytes;  // X slice + two reduction buffers
 }
 }  // namespace gemv
 
@@ -1016,27 +1016,29 @@ __global__ void __launch_bounds__(gemv::kThreads) w4a16_gemv_kernel(
   const int nkb = (K + kKB - 1) / kKB;
   const int kb0 = rank * kb_per;
   const int nloc = max(0, min(kb_per, nkb - kb0));  // k-blocks of this slice
-  const int row_cta = static_cast<int>(blockIdx.y) * kRowsCta;
+  const int n_tiles = (N + kRowsCta - 1) / kRowsCta;
   const int64_t row_bytes = K / 2, groups_per_row = K / 64;
   constexpr int kMsz = MT == kF32 ? 4 : 2;
   const uint8_t* sc_base = static_cast<const uint8_t*>(args.scale);
   const uint8_t* zr_base = static_cast<const uint8_t*>(args.zero);
 
-  // this lane's n-tile rows (8r + g of the warp's 16) at the slice start: code and meta
-  // pointers; invalid rows read nothing (codes and meta 0 -> W' = +0)
+  // this lane's n-tile rows (8r + g of the warp's 16) of row tile `tile` at the slice start:
+  // code and meta pointers; invalid rows read nothing (codes and meta 0 -> W' = +0)
   const uint8_t* crow[kNT];
   const uint8_t* srow[kNT];
   const uint8_t* zrow[kNT];
   bool rin[kNT];
+  auto set_rows = [&](int tile) {
 #pragma unroll
-  for (int r = 0; r < kNT; ++r) {
-    const int row = row_cta + warp * (kNT * 8) + 8 * r + g;
-    rin[r] = row < N;
-    crow[r] = packed + row * row_bytes + static_cast<int64_t>(kb0) * 64 + 16 * t;
-    const int64_t gi = row * groups_per_row + 2 * static_cast<int64_t>(kb0) + (t >> 1);
-    srow[r] = sc_base + gi * kMsz;
-    zrow[r] = zr_base + gi * kMsz;
-  }
+    for (int r = 0; r < kNT; ++r) {
+      const int row = tile * kRowsCta + warp * (kNT * 8) + 8 * r + g;
+      rin[r] = row < N;
+      crow[r] = packed + row * row_bytes + static_cast<int64_t>(kb0) * 64 + 16 * t;
+      const int64_t gi = row * groups_per_row + 2 * static_cast<int64_t>(kb0) + (t >> 1);
+      srow[r] = sc_base + gi * kMsz;
+      zrow[r] = zr_base + gi * kMsz;
+    }
+  };
 
   uint4 code[kDepth][kNT];
   uint32_t msc[kDepth][kNT], mzr[kDepth][kNT];
@@ -1055,18 +1057,25 @@ __global__ void __launch_bounds__(gemv::kThreads) w4a16_gemv_kernel(
       }
     }
   };
+  auto load_first = [&]() {
+#pragma unroll
+    for (int i = 0; i < kDepth; ++i)
+      if (i < nloc) load_kb(i, code[i], msc[i], mzr[i]);
+  };
+
   // Programmatic dependent launch (HQQ_FLAG_OVERLAP_WEIGHTS): the next kernel on the stream
   // may start now; this one loads its weight codes and meta (which no earlier work writes, by
   // the flag's promise) and then waits for the previous kernel's completion and memory before
   // it reads X or writes anything. Without the launch attribute both are no-ops.
+  int tile = static_cast<int>(blockIdx.y);
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < kDepth; ++i)
-    if (i < nloc) load_kb(i, code[i], msc[i], mzr[i]);
+  set_rows(tile);
+  load_first();
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // X[0..15][slice] -> shared memory: 16-byte piece q (k = 8q within the slice) of token m at
-  // m * rs + (q / 16) * 256 + (q % 4) * 64 + ((q / 4) % 4) * 16; zeros past M and past K
+  // X[0..15][slice] -> shared memory, once for every row tile of this CTA: 16-byte piece q
+  // (k = 8q within the slice) of token m at m * rs + (q / 16) * 256 + (q % 4) * 64 +
+  // ((q / 4) % 4) * 16; zeros past M and past K
   const uint32_t rs = x_row_bytes(kb_per);
   {
     // asynchronous 16-byte copies (all issued before one wait; 0 source bytes = zero fill);
@@ -1090,80 +1099,98 @@ __global__ void __launch_bounds__(gemv::kThreads) w4a16_gemv_kernel(
   }
   __syncthreads();
 
-  float acc[kNT][4];
-#pragma unroll
-  for (int r = 0; r < kNT; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
   const uint8_t* xa_row = smem + g * rs + t * 16;
   const uint8_t* xb_row = smem + (g + 8) * rs + t * 16;
+  const int S = 1 << lg_s, lg_rpo = kLgRowsCta - lg_s, rpo = kRowsCta >> lg_s;
+  typedef typename std::conditional<F16, __half, __nv_bfloat16>::type T;
+  const unsigned short* bias = reinterpret_cast<const unsigned short*>(args.bias);
 
-  for (int base = 0; base < nloc; base += kDepth) {
+  // Row tiles blockIdx.y, blockIdx.y + gridDim.y, ... (the same sequence in every CTA of the
+  // cluster, so all of them take the same barriers). The reduction slots alternate between
+  // two buffers: a tile's partial sums are written after the barrier that ends the previous
+  // tile, and its buffer is written again only two tiles later, after the barrier that the
+  // owner passes once it has read it.
+  for (int it = 0; tile < n_tiles; tile += static_cast<int>(gridDim.y), ++it) {
+    float acc[kNT][4];
 #pragma unroll
-    for (int d = 0; d < kDepth; ++d) {
-      const int i = base + d;
-      if (i < nloc) {
-        float2 nz2[kNT], sc2[kNT];
+    for (int r = 0; r < kNT; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
+
+    for (int base = 0; base < nloc; base += kDepth) {
 #pragma unroll
-        for (int r = 0; r < kNT; ++r) {
-          const float sc = meta_f32<MT>(msc[d][r]), z = meta_f32<MT>(mzr[d][r]);
-          nz2[r] = make_float2(-z, -z);
-          sc2[r] = make_float2(sc, sc);
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          // word j: k = 32t + 8j .. +7 -> steps 2j (k +0..3) and 2j+1 (k +4..7)
-          const uint4 xa = *reinterpret_cast<const uint4*>(xa_row + i * 256 + j * 64);
-          const uint4 xb = *reinterpret_cast<const uint4*>(xb_row + i * 256 + j * 64);
+      for (int d = 0; d < kDepth; ++d) {
+        const int i = base + d;
+        if (i < nloc) {
+          float2 nz2[kNT], sc2[kNT];
 #pragma unroll
           for (int r = 0; r < kNT; ++r) {
-            const uint32_t w = j == 0 ? code[d][r].x : j == 1 ? code[d][r].y
-                             : j == 2 ? code[d][r].z : code[d][r].w;
-            const uint4 o = dequant8<F16>(w, nz2[r], sc2[r]);
-            mma_16816<F16>(acc[r], xa.x, xb.x, xa.y, xb.y, o.x, o.y);
-            mma_16816<F16>(acc[r], xa.z, xb.z, xa.w, xb.w, o.z, o.w);
+            const float sc = meta_f32<MT>(msc[d][r]), z = meta_f32<MT>(mzr[d][r]);
+            nz2[r] = make_float2(-z, -z);
+            sc2[r] = make_float2(sc, sc);
           }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            // word j: k = 32t + 8j .. +7 -> steps 2j (k +0..3) and 2j+1 (k +4..7)
+            const uint4 xa = *reinterpret_cast<const uint4*>(xa_row + i * 256 + j * 64);
+            const uint4 xb = *reinterpret_cast<const uint4*>(xb_row + i * 256 + j * 64);
+#pragma unroll
+            for (int r = 0; r < kNT; ++r) {
+              const uint32_t w = j == 0 ? code[d][r].x : j == 1 ? code[d][r].y
+                               : j == 2 ? code[d][r].z : code[d][r].w;
+              const uint4 o = dequant8<F16>(w, nz2[r], sc2[r]);
+              mma_16816<F16>(acc[r], xa.x, xb.x, xa.y, xb.y, o.x, o.y);
+              mma_16816<F16>(acc[r], xa.z, xb.z, xa.w, xb.w, o.z, o.w);
+            }
+          }
+          if (i + kDepth < nloc) load_kb(i + kDepth, code[d], msc[d], mzr[d]);
         }
-        if (i + kDepth < nloc) load_kb(i + kDepth, code[d], msc[d], mzr[d]);
       }
     }
-  }
 
-  // partial sums -> the owner CTA's slot for this rank: red[(src * RPO + row_local) * 16 + m]
-  const int S = 1 << lg_s, lg_rpo = kLgRowsCta - lg_s, rpo = kRowsCta >> lg_s;
-  const uint32_t red_local = smem_u32(smem + 16 * rs);
-#pragma unroll
-  for (int r = 0; r < kNT; ++r) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int rho = warp * (kNT * 8) + 8 * r + 2 * t + (e & 1);
-      const int m = g + 8 * (e >> 1);
-      const int owner = rho >> lg_rpo, rl = rho & (rpo - 1);
-      const uint32_t off = static_cast<uint32_t>(((rank * rpo + rl) * 16 + m) * 4);
-      st_cluster_f32(cluster_addr(red_local + off, static_cast<uint32_t>(owner)), acc[r][e]);
+    // the next tile's first codes are in flight while this tile is reduced
+    const int row_cta = tile * kRowsCta;
+    if (tile + static_cast<int>(gridDim.y) < n_tiles) {
+      set_rows(tile + static_cast<int>(gridDim.y));
+      load_first();
     }
-  }
-  cluster_sync();
 
-  // owner: rows row_cta + rank * rpo .. + rpo - 1, every token < M, two rows per store
-  typedef typename std::conditional<F16, __half, __nv_bfloat16>::type T;
-  const float* red = reinterpret_cast<const float*>(smem + 16 * rs);
-  const unsigned short* bias = reinterpret_cast<const unsigned short*>(args.bias);
-  const int nbase = row_cta + rank * rpo;
-  for (int idx = threadIdx.x; idx < (M << (lg_rpo - 1)); idx += kThreads) {
-    const int m = idx >> (lg_rpo - 1), pr = 2 * (idx & ((rpo >> 1) - 1));
-    if (nbase + pr >= N) continue;
-    float v0 = 0.0f, v1 = 0.0f;
-    for (int src = 0; src < S; ++src) {  // fixed order
-      v0 = __fadd_rn(v0, red[(src * rpo + pr) * 16 + m]);
-      v1 = __fadd_rn(v1, red[(src * rpo + pr + 1) * 16 + m]);
+    // partial sums -> the owner CTA's slot for this rank:
+    // red[(src * RPO + row_local) * 16 + m], buffer it & 1
+    const uint32_t red_local = smem_u32(smem + 16 * rs + (it & 1) * kRedBytes);
+#pragma unroll
+    for (int r = 0; r < kNT; ++r) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int rho = warp * (kNT * 8) + 8 * r + 2 * t + (e & 1);
+        const int m = g + 8 * (e >> 1);
+        const int owner = rho >> lg_rpo, rl = rho & (rpo - 1);
+        const uint32_t off = static_cast<uint32_t>(((rank * rpo + rl) * 16 + m) * 4);
+        st_cluster_f32(cluster_addr(red_local + off, static_cast<uint32_t>(owner)), acc[r][e]);
+      }
     }
-    if (bias != nullptr) {
-      v0 = __fadd_rn(v0, F16 ? f16_bits_to_f32(bias[nbase + pr]) : bf16_bits_to_f32(bias[nbase + pr]));
-      v1 = __fadd_rn(v1, F16 ? f16_bits_to_f32(bias[nbase + pr + 1])
-                             : bf16_bits_to_f32(bias[nbase + pr + 1]));
+    cluster_sync();
+
+    // owner: rows row_cta + rank * rpo .. + rpo - 1, every token < M, two rows per store
+    const float* red = reinterpret_cast<const float*>(smem + 16 * rs + (it & 1) * kRedBytes);
+    const int nbase = row_cta + rank * rpo;
+    for (int idx = threadIdx.x; idx < (M << (lg_rpo - 1)); idx += kThreads) {
+      const int m = idx >> (lg_rpo - 1), pr = 2 * (idx & ((rpo >> 1) - 1));
+      if (nbase + pr >= N) continue;
+      float v0 = 0.0f, v1 = 0.0f;
+      for (int src = 0; src < S; ++src) {  // fixed order
+        v0 = __fadd_rn(v0, red[(src * rpo + pr) * 16 + m]);
+        v1 = __fadd_rn(v1, red[(src * rpo + pr + 1) * 16 + m]);
+      }
+      if (bias != nullptr) {
+        v0 = __fadd_rn(v0, F16 ? f16_bits_to_f32(bias[nbase + pr]) : bf16_bits_to_f32(bias[nbase + pr]));
+        v1 = __fadd_rn(v1, F16 ? f16_bits_to_f32(bias[nbase + pr + 1])
+                               : bf16_bits_to_f32(bias[nbase + pr + 1]));
+      }
+      *reinterpret_cast<uint32_t*>(reinterpret_cast<T*>(args.Y) + static_cast<int64_t>(m) * N +
+                                   nbase + pr) = pack2_16<F16 ? kF16 : kBF16>(v0, v1);
     }
-    *reinterpret_cast<uint32_t*>(reinterpret_cast<T*>(args.Y) + static_cast<int64_t>(m) * N +
-                                 nbase + pr) = pack2_16<F16 ? kF16 : kBF16>(v0, v1);
   }
+  // No remote write follows the last barrier (each CTA then reads only its own slots), so
+  // the CTAs of the cluster may leave independently.
 }
 
 // ---------------------------------------------------------------- host side
@@ -1194,6 +1221,34 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const void* b
   return encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Clusters of S CTAs of `kernel` with `smem` bytes of dynamic shared memory that fit on the
+// device at once (0 if the runtime cannot tell); cached per (kernel, S, smem).
+int gemv_resident_clusters(const void* kernel, int S, uint32_t smem, const cudaLaunchConfig_t* cfg) {
+  struct Entry { const void* k; int s; uint32_t smem; int n; };
+  static std::mutex mu;
+  static Entry cache[64];
+  static int used = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].k == kernel && cache[i].s == S && cache[i].smem == smem) return cache[i].n;
+  cudaLaunchConfig_t c = *cfg;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = static_cast<unsigned>(S);
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  c.attrs = at;
+  c.numAttrs = 1;
+  c.gridDim = dim3(static_cast<unsigned>(S), 1, 1);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &c) != cudaSuccess) {
+    (void)cudaGetLastError();  // an unanswered query only means one cluster per row tile
+    n = 0;
+  }
+  if (used < 64) cache[used++] = Entry{kernel, S, smem, n};
+  return n;
 }
 
 template <bool F16, int MT>
@@ -1229,11 +1284,16 @@ cudaError_t launch_typed(const GemmJob& job, cudaStream_t stream) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(gemv::smem_bytes(gemv::kMaxKbPerSlice)));
     if (e != cudaSuccess) return e;
-    cfg.gridDim = dim3(static_cast<unsigned>(S),
-                       static_cast<unsigned>((job.N + gemv::kRowsCta - 1) / gemv::kRowsCta));
+    const int64_t tiles = (job.N + gemv::kRowsCta - 1) / gemv::kRowsCta;
     cfg.blockDim = dim3(gemv::kThreads);
     cfg.dynamicSmemBytes = smem;
     attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    // one wave of clusters, each looping over row tiles: at most as many clusters as fit on
+    // the GPU at once (X is staged once per CTA, the next tile's codes load during a reduction)
+    const int resident = gemv_resident_clusters(
+        reinterpret_cast<const void*>(&w4a16_gemv_kernel<F16, MT>), S, smem, &cfg);
+    const int64_t ny = resident > 0 && tiles > resident ? resident : tiles;
+    cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(ny));
     if (job.overlap_weights) cfg.numAttrs = 2;  // the decode kernel waits before reading X
     const uint8_t* packed = job.packed;
     const int lg_s = S == 8 ? 3 : S == 4 ? 2 : S == 2 ? 1 : 0;
