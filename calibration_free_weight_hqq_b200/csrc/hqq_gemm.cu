@@ -962,23 +962,38 @@ __global__ void __launch_bounds__(skinny::kThreads, 2)
 #ifndef HQQ_GEMV_DEPTH
 #define HQQ_GEMV_DEPTH 4
 #endif
+// When the next kernel on the stream may launch (HQQ_FLAG_OVERLAP_WEIGHTS): 1 = after this
+// kernel's last tile, 0 = at entry. At entry the dependent's persistent grid, sized for an idle
+// GPU, started partly late and its clusters then carried several tiles each (measured slower).
+#ifndef HQQ_GEMV_TRIGGER_LATE
+#define HQQ_GEMV_TRIGGER_LATE 1
+#endif
 
 namespace gemv {
-constexpr int kWarps = HQQ_GEMV_WARPS;
-constexpr int kThreads = 32 * kWarps;
-constexpr int kNT = HQQ_GEMV_NT;             // n-tiles (8 W' rows) per warp
-constexpr int kRowsCta = kWarps * kNT * 8;   // 128
-constexpr int kLgRowsCta = kRowsCta == 256 ? 8 : kRowsCta == 128 ? 7 : kRowsCta == 64 ? 6 : 5;
-static_assert((1 << kLgRowsCta) == kRowsCta, "power-of-two CTA rows");
 constexpr int kKB = 128;                     // k per k-block
 constexpr int kDepth = HQQ_GEMV_DEPTH;       // k-blocks of codes in flight per warp
 constexpr int kMaxKbPerSlice = 32;           // X tile <= 16 x 8256 B
 constexpr int kMaxM = 16;
-constexpr uint32_t kRedBytes = kRowsCta * 16 * 4;
 __host__ __device__ constexpr uint32_t x_row_bytes(int kb_per) { return kb_per * 256 + 64; }
-__host__ __device__ constexpr uint32_t smem_bytes(int kb_per) {
-  return 16 * x_row_bytes(kb_per) + 2 * kRedBytes;  // X slice + two reduction buffers
-}
+// Tile shape: WARPS warps of NT n-tiles (8 W' rows each) per CTA.
+template <int WARPS, int NT>
+struct Shape {
+  static constexpr int kWarps = WARPS;
+  static constexpr int kThreads = 32 * WARPS;
+  static constexpr int kNT = NT;
+  static constexpr int kRowsCta = WARPS * NT * 8;
+  static constexpr int kLgRowsCta =
+      kRowsCta == 256 ? 8 : kRowsCta == 128 ? 7 : kRowsCta == 64 ? 6 : 5;
+  static_assert((1 << kLgRowsCta) == kRowsCta, "power-of-two CTA rows");
+  static constexpr uint32_t kRedBytes = kRowsCta * 16 * 4;
+  static constexpr uint32_t smem_bytes(int kb_per) {
+    return 16 * x_row_bytes(kb_per) + 2 * kRedBytes;  // X slice + two reduction buffers
+  }
+};
+// The shapes built: 128-row tiles (the default), and 64-row tiles for layers so wide that the
+// 128-row tiles outnumber the clusters that fit at once.
+using Wide = Shape<HQQ_GEMV_WARPS, HQQ_GEMV_NT>;
+using Narrow = Shape<4, 2>;
 }  // namespace gemv
 
 template <bool F16>
@@ -1003,11 +1018,16 @@ __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
 
 // grid (S, ceil(N / 128)), cluster (S, 1, 1) with S = 2^lg_s; kb_per = k-blocks per slice;
 // M <= 16.
-template <bool F16, int MT>
-__global__ void __launch_bounds__(gemv::kThreads) w4a16_gemv_kernel(
+template <bool F16, int MT, int WARPS, int NT>
+__global__ void __launch_bounds__(32 * WARPS) w4a16_gemv_kernel(
     const void* __restrict__ X, const uint8_t* __restrict__ packed, const GemmArgs args,
     int lg_s, int kb_per) {
   using namespace gemv;
+  using Sh = Shape<WARPS, NT>;
+  constexpr int kWarps = Sh::kWarps, kThreads = Sh::kThreads, kNT = Sh::kNT;
+  constexpr int kRowsCta = Sh::kRowsCta, kLgRowsCta = Sh::kLgRowsCta;
+  constexpr uint32_t kRedBytes = Sh::kRedBytes;
+  (void)kWarps;
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -1063,12 +1083,14 @@ __global__ void __launch_bounds__(gemv::kThreads) w4a16_gemv_kernel(
       if (i < nloc) load_kb(i, code[i], msc[i], mzr[i]);
   };
 
-  // Programmatic dependent launch (HQQ_FLAG_OVERLAP_WEIGHTS): the next kernel on the stream
-  // may start now; this one loads its weight codes and meta (which no earlier work writes, by
-  // the flag's promise) and then waits for the previous kernel's completion and memory before
-  // it reads X or writes anything. Without the launch attribute both are no-ops.
+  // Programmatic dependent launch (HQQ_FLAG_OVERLAP_WEIGHTS): this kernel may start before the
+  // previous one on the stream has finished; it loads its weight codes and meta (which no
+  // earlier work writes, by the flag's promise) and then waits for the previous kernel's
+  // completion and memory before it reads X or writes anything. It lets the next kernel
+  // launch once its own tiles are done (HQQ_GEMV_TRIGGER_LATE). Without the launch attribute
+  // these instructions are no-ops.
   int tile = static_cast<int>(blockIdx.y);
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (!HQQ_GEMV_TRIGGER_LATE) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   set_rows(tile);
   load_first();
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1191,6 +1213,7 @@ __global__ void __launch_bounds__(gemv::kThreads) w4a16_gemv_kernel(
   }
   // No remote write follows the last barrier (each CTA then reads only its own slots), so
   // the CTAs of the cluster may leave independently.
+  if (HQQ_GEMV_TRIGGER_LATE) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- host side
@@ -1223,9 +1246,9 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const void* b
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Clusters of S CTAs of `kernel` with `smem` bytes of dynamic shared memory that fit on the
-// device at once (0 if the runtime cannot tell); cached per (kernel, S, smem).
-int gemv_resident_clusters(const void* kernel, int S, uint32_t smem, const cudaLaunchConfig_t* cfg) {
+// Clusters of S CTAs of `kernel` (`threads` a CTA, `smem` bytes of dynamic shared memory)
+// that fit on the device at once (0 if the runtime cannot tell); cached per (kernel, S, smem).
+int gemv_resident_clusters(const void* kernel, int S, uint32_t smem, int threads) {
   struct Entry { const void* k; int s; uint32_t smem; int n; };
   static std::mutex mu;
   static Entry cache[64];
@@ -1233,7 +1256,7 @@ int gemv_resident_clusters(const void* kernel, int S, uint32_t smem, const cudaL
   std::lock_guard<std::mutex> lock(mu);
   for (int i = 0; i < used; ++i)
     if (cache[i].k == kernel && cache[i].s == S && cache[i].smem == smem) return cache[i].n;
-  cudaLaunchConfig_t c = *cfg;
+  cudaLaunchConfig_t c = {};
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = static_cast<unsigned>(S);
@@ -1242,6 +1265,8 @@ int gemv_resident_clusters(const void* kernel, int S, uint32_t smem, const cudaL
   c.attrs = at;
   c.numAttrs = 1;
   c.gridDim = dim3(static_cast<unsigned>(S), 1, 1);
+  c.blockDim = dim3(static_cast<unsigned>(threads));
+  c.dynamicSmemBytes = smem;
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, kernel, &c) != cudaSuccess) {
     (void)cudaGetLastError();  // an unanswered query only means one cluster per row tile
@@ -1249,6 +1274,33 @@ int gemv_resident_clusters(const void* kernel, int S, uint32_t smem, const cudaL
   }
   if (used < 64) cache[used++] = Entry{kernel, S, smem, n};
   return n;
+}
+
+template <bool F16, int MT, typename Sh>
+cudaError_t set_gemv_smem() {
+  return cudaFuncSetAttribute(w4a16_gemv_kernel<F16, MT, Sh::kWarps, Sh::kNT>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(Sh::smem_bytes(gemv::kMaxKbPerSlice)));
+}
+
+// The decode kernel with tile shape Sh: one wave of clusters, each looping over row tiles.
+template <bool F16, int MT, typename Sh>
+cudaError_t launch_gemv(const GemmJob& job, const GemmArgs& a, cudaLaunchConfig_t* cfg, int S,
+                        int lg_s, int kb_per) {
+  cudaError_t e = set_gemv_smem<F16, MT, Sh>();
+  if (e != cudaSuccess) return e;
+  const uint32_t smem = Sh::smem_bytes(kb_per);
+  const int64_t tiles = (job.N + Sh::kRowsCta - 1) / Sh::kRowsCta;
+  const int resident = gemv_resident_clusters(
+      reinterpret_cast<const void*>(&w4a16_gemv_kernel<F16, MT, Sh::kWarps, Sh::kNT>), S, smem,
+      Sh::kThreads);
+  const int64_t ny = resident > 0 && tiles > resident ? resident : tiles;
+  cfg->blockDim = dim3(Sh::kThreads);
+  cfg->dynamicSmemBytes = smem;
+  cfg->gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(ny));
+  const uint8_t* packed = job.packed;
+  return cudaLaunchKernelEx(cfg, w4a16_gemv_kernel<F16, MT, Sh::kWarps, Sh::kNT>, job.X, packed,
+                            a, lg_s, kb_per);
 }
 
 template <bool F16, int MT>
@@ -1278,26 +1330,21 @@ cudaError_t launch_typed(const GemmJob& job, cudaStream_t stream) {
   const int S = nkb >= 16 ? 8 : nkb >= 8 ? 4 : nkb >= 4 ? 2 : 1;
   const int kb_per = (nkb + S - 1) / S;
   if (job.M <= gemv::kMaxM && kb_per <= gemv::kMaxKbPerSlice &&
-      (job.N + gemv::kRowsCta - 1) / gemv::kRowsCta <= 65535) {
-    const uint32_t smem = gemv::smem_bytes(kb_per);
-    cudaError_t e = cudaFuncSetAttribute(w4a16_gemv_kernel<F16, MT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(gemv::smem_bytes(gemv::kMaxKbPerSlice)));
-    if (e != cudaSuccess) return e;
-    const int64_t tiles = (job.N + gemv::kRowsCta - 1) / gemv::kRowsCta;
-    cfg.blockDim = dim3(gemv::kThreads);
-    cfg.dynamicSmemBytes = smem;
+      (job.N + gemv::Narrow::kRowsCta - 1) / gemv::Narrow::kRowsCta <= 65535) {
     attr[0].val.clusterDim.x = static_cast<unsigned>(S);
-    // one wave of clusters, each looping over row tiles: at most as many clusters as fit on
-    // the GPU at once (X is staged once per CTA, the next tile's codes load during a reduction)
-    const int resident = gemv_resident_clusters(
-        reinterpret_cast<const void*>(&w4a16_gemv_kernel<F16, MT>), S, smem, &cfg);
-    const int64_t ny = resident > 0 && tiles > resident ? resident : tiles;
-    cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(ny));
     if (job.overlap_weights) cfg.numAttrs = 2;  // the decode kernel waits before reading X
-    const uint8_t* packed = job.packed;
     const int lg_s = S == 8 ? 3 : S == 4 ? 2 : S == 2 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, w4a16_gemv_kernel<F16, MT>, job.X, packed, a, lg_s, kb_per);
+    // 128-row tiles when one wave of clusters covers the rows (or nearly), 64-row tiles for
+    // wider layers (measured: the 11008-row layers 30.7 -> 26.6 us, the 4096-row ones slower)
+    const int64_t wide_tiles = (job.N + gemv::Wide::kRowsCta - 1) / gemv::Wide::kRowsCta;
+    cudaError_t e = set_gemv_smem<F16, MT, gemv::Wide>();
+    if (e != cudaSuccess) return e;
+    const int wide_resident = gemv_resident_clusters(
+        reinterpret_cast<const void*>(&w4a16_gemv_kernel<F16, MT, gemv::Wide::kWarps, gemv::Wide::kNT>),
+        S, gemv::Wide::smem_bytes(kb_per), gemv::Wide::kThreads);
+    if (wide_resident > 0 && wide_tiles > wide_resident)
+      return launch_gemv<F16, MT, gemv::Narrow>(job, a, &cfg, S, lg_s, kb_per);
+    return launch_gemv<F16, MT, gemv::Wide>(job, a, &cfg, S, lg_s, kb_per);
   }
   if (job.M <= skinny::kMaxM) {
     const int ntok = static_cast<int>(

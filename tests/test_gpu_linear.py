@@ -312,3 +312,22 @@ def test_linear_decode_overlap_flag_keeps_every_dependency():
     for Y in (Y1, Y2):
         assert np.array_equal(Y.float().cpu().numpy(), Wd[:, ks].T)
     assert_no_timeouts()
+
+
+def test_linear_decode_wide_layer_one_hot():
+    """A layer wide enough that its 128-row tiles outnumber the clusters that fit on the GPU
+    (11008 rows) runs the decode kernel with 64-row tiles, each cluster looping over several;
+    one-hot rows make every output one dequantized weight: exact for every row tile."""
+    N, K, M = 11008, 2112, 16
+    codes, scale, zero, dev = make_layer(N, K, 4242)
+    ks = 131 * np.arange(M) + 7
+    X = torch.zeros(M, K, dtype=torch.bfloat16)
+    X[torch.arange(M), torch.from_numpy(ks)] = 1.0
+    for flag in (False, True):
+        p = hqq.make_params(4, 64, 1, w_dtype=torch.bfloat16, meta_dtype=torch.bfloat16,
+                            overlap_weights=flag)
+        Y = hqq.hqq_linear(X.cuda(), dev["packed"], dev["scale"], dev["zero"], N, p)
+        torch.cuda.synchronize()
+        Wd = oracle.round_to_dtype(oracle.dequantize(codes, scale, zero, N, K, 64, 1), "bf16")
+        assert np.array_equal(Y.float().cpu().numpy(), Wd[:, ks].T)
+    assert_no_timeouts()
