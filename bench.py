@@ -516,8 +516,8 @@ def run_linear(hqq, dev, args, tokens: int = 4096):
                       "of up to 8 CTAs)",
             "timing": "CUDA graph of the 7 launches, L2 flushed before each replay",
             "ms_per_step": round(ms_dec, 4), "launches_per_step": len(dec),
-            "overlap": "HQQ_FLAG_OVERLAP_WEIGHTS (programmatic dependent launch: a layer's "
-                       "weight codes load while the previous layer finishes)",
+            "overlap": "HQQ_FLAG_OVERLAP_WEIGHTS (programmatic dependent launch: a layer may "
+                       "start, and load its weight codes, before the previous layer finishes)",
             "ms_per_step_without_overlap": round(ms_dec_plain, 4),
             "cublas_bf16_weight_ms_per_step": round(ms_dec_cublas, 4),
             "tflops": round(sum(2.0 * dec_tokens * m.rows * m.cols for m, *_ in dec)
