@@ -242,6 +242,12 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
@@ -278,9 +284,12 @@ __device__ __forceinline__ bool mbar_wait_cl(uint32_t bar, uint32_t parity,
     }
   }
 }
+// Arrive on a barrier of the peer CTA. The default semantics (release at CTA scope) suffice for
+// a "your operand half is written" signal: the data it announces is the peer's own shared
+// memory, complete before this thread acquired its local barrier. A cluster-scope release
+// measured about 0.9 us per arrive on B200 when one is relayed per k-block.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 // TMA load whose completion is counted on a barrier of either CTA of the pair.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x,
@@ -965,6 +974,11 @@ __global__ void __launch_bounds__(skinny::kThreads, 2)
 // When the next kernel on the stream may launch (HQQ_FLAG_OVERLAP_WEIGHTS): 1 = after this
 // kernel's last tile, 0 = at entry. At entry the dependent's persistent grid, sized for an idle
 // GPU, started partly late and its clusters then carried several tiles each (measured slower).
+// Where the next row tile's first code loads are issued: 1 = between the arrive and the wait of
+// the tile's cluster barrier, 0 = before the barrier.
+#ifndef HQQ_GEMV_SPLIT_SYNC
+#define HQQ_GEMV_SPLIT_SYNC 1
+#endif
 #ifndef HQQ_GEMV_TRIGGER_LATE
 #define HQQ_GEMV_TRIGGER_LATE 1
 #endif
@@ -1168,12 +1182,13 @@ __global__ void __launch_bounds__(32 * WARPS) w4a16_gemv_kernel(
       }
     }
 
-    // the next tile's first codes are in flight while this tile is reduced
     const int row_cta = tile * kRowsCta;
+#if !HQQ_GEMV_SPLIT_SYNC
     if (tile + static_cast<int>(gridDim.y) < n_tiles) {
       set_rows(tile + static_cast<int>(gridDim.y));
       load_first();
     }
+#endif
 
     // partial sums -> the owner CTA's slot for this rank:
     // red[(src * RPO + row_local) * 16 + m], buffer it & 1
@@ -1189,7 +1204,19 @@ __global__ void __launch_bounds__(32 * WARPS) w4a16_gemv_kernel(
         st_cluster_f32(cluster_addr(red_local + off, static_cast<uint32_t>(owner)), acc[r][e]);
       }
     }
+#if HQQ_GEMV_SPLIT_SYNC
+    // The barrier's release orders this thread's earlier loads too, so the next tile's first
+    // codes are requested after the arrive: they are in flight during the wait and the
+    // reduction instead of delaying the arrive until they return.
+    cluster_arrive();
+    if (tile + static_cast<int>(gridDim.y) < n_tiles) {
+      set_rows(tile + static_cast<int>(gridDim.y));
+      load_first();
+    }
+    cluster_wait();
+#else
     cluster_sync();
+#endif
 
     // owner: rows row_cta + rank * rpo .. + rpo - 1, every token < M, two rows per store
     const float* red = reinterpret_cast<const float*>(smem + 16 * rs + (it & 1) * kRedBytes);
