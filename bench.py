@@ -376,12 +376,16 @@ def capture_graph(fn):
 
 
 def time_graph(graph, warmup: int, steps: int, flush) -> float:
-    """Median device time (ms) of one replay, L2 flushed (flush buffer written) before each."""
+    """Device time (ms) of one replay, L2 flushed (flush buffer written) before each: the mean
+    of the per-replay CUDA-event times after dropping the fastest and slowest 10 %. Event times
+    on B200 come in steps of 2.048 us, so a median of a short launch is quantized to that step;
+    the trimmed mean of at least 20 replays resolves differences below it and still ignores
+    outliers."""
     for _ in range(warmup):
         graph.replay()
     torch.cuda.synchronize()
     per = []
-    for _ in range(steps):
+    for _ in range(max(steps, 20)):
         flush.fill_(1)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
@@ -389,7 +393,10 @@ def time_graph(graph, warmup: int, steps: int, flush) -> float:
         b.record()
         torch.cuda.synchronize()
         per.append(a.elapsed_time(b))
-    return statistics.median(per)
+    per.sort()
+    cut = len(per) // 10
+    kept = per[cut:len(per) - cut]
+    return sum(kept) / len(kept)
 
 
 def run_linear(hqq, dev, args, tokens: int = 4096):
@@ -923,6 +930,12 @@ SINGLE_CASES = {
     "quantize_3b_g64": (16384, 8192, "bf16", 3, 64, 1),
     "quantize_fp16_4096x1024": (4096, 1024, "f16", 4, 64, 1),
 }
+# dequantize with 8-bit second-level scale/zero (runs of 128), the layouts of the 70B MLP
+# workload's two matrices, on a [16384, 8192] bf16 weight
+SINGLE_DEQ_META = {
+    "dequantize_3b_g64_meta8": (16384, 8192, 3, 64),
+    "dequantize_1b_g32_meta8": (16384, 8192, 1, 32),
+}
 
 
 def single_dequantize_block(reps: int = 10):
@@ -955,11 +968,43 @@ def single_dequantize_block(reps: int = 10):
             "GB_per_s_algorithmic": round(gbs, 1), "hbm_frac": round(gbs / peaks()["hbm_gbs"], 4)}
 
 
+def single_dequantize_meta(kind: str, reps: int = 10):
+    """One matrix of SINGLE_DEQ_META[kind], quantized with 8-bit scale and zero, dequantized to
+    bf16 `reps` times after warm-up (hqq_dequantize_ex)."""
+    import calibration_free_weight_hqq_b200 as hqq
+    from calibration_free_weight_hqq_b200 import synthetic
+    rows, cols, nbits, G = SINGLE_DEQ_META[kind]
+    W = synthetic.weight(rows, cols, seed=5, dtype=torch.bfloat16, device="cuda")
+    params = hqq.make_params(nbits, G, 1, w_dtype=torch.bfloat16, quant_scale=True,
+                             quant_zero=True, meta_group_size=128)
+    q = hqq.hqq_quantize_ex(W, params)
+    D = torch.empty_like(W)
+    for _ in range(2):
+        hqq.hqq_dequantize_ex(q, rows, cols, params, out=D)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        hqq.hqq_dequantize_ex(q, rows, cols, params, out=D)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    n = rows * cols
+    ng = n // G
+    runs = -(-ng // 128)
+    nbytes = hqq.hqq_packed_bytes(rows, cols, nbits) + 2 * ng + 2 * runs * 8 + 2 * n
+    return {"single": kind, "shape": [rows, cols], "nbits": nbits, "group_size": G,
+            "ms": round(ms, 4), "GB_per_s": round(nbytes / ms / 1e6, 1),
+            "hbm_frac": round(nbytes / ms / 1e6 / peaks()["hbm_gbs"], 4)}
+
+
 def single(kind: str, reps: int = 10):
     """One matrix of SINGLE_CASES[kind]: time `reps` solver or dequantize launches after
     warm-up (the cases the ncu captures in profiles/ use)."""
     import calibration_free_weight_hqq_b200 as hqq
     from calibration_free_weight_hqq_b200 import synthetic
+    if kind in SINGLE_DEQ_META:
+        return single_dequantize_meta(kind, reps)
     rows, cols, dt, nbits, G, axis = SINGLE_CASES[kind]
     dtype = torch.float16 if dt == "f16" else torch.bfloat16
     W = synthetic.weight(rows, cols, seed=5, dtype=dtype, device="cuda")
@@ -1007,10 +1052,10 @@ def main():
                     help="leave the four smaller configurations out of the JSON line")
     ap.add_argument("--mixed", action="store_true",
                     help="whole model with per-layer configurations (8/4/2 bits) and exit")
-    ap.add_argument("--single", choices=sorted(SINGLE_CASES) + ["dequantize_block_batched",
-                                                                 "linear", "decode"],
-                    help="time one matrix of a profiling case (SINGLE_CASES), one 4096^3 "
-                         "linear layer, or one 4096x4096 layer at 16 tokens, and exit")
+    ap.add_argument("--single", choices=sorted(SINGLE_CASES) + sorted(SINGLE_DEQ_META) +
+                    ["dequantize_block_batched", "linear", "decode"],
+                    help="time one matrix of a profiling case (SINGLE_CASES, SINGLE_DEQ_META), "
+                         "one 4096^3 linear layer, or one 4096x4096 layer at 16 tokens, and exit")
     args = ap.parse_args()
     if args.configs:
         for line in configs_table():

@@ -214,7 +214,10 @@ __device__ __forceinline__ void store1(void* out, int64_t k, float v) {
 // Any nbits, plain or second-level meta, any output type. A tile (kDTile1 elements, a multiple
 // of every group size) starts on a group and on a byte of the code stream, so its 64-bit
 // bases are formed once and the per-chunk index work is 32-bit.
-constexpr int kD1Unroll = 4;
+#ifndef HQQ_DQ1_UNROLL
+#define HQQ_DQ1_UNROLL 4
+#endif
+constexpr int kD1Unroll = HQQ_DQ1_UNROLL;
 constexpr int kDTile1 = kDBlock * 8 * kD1Unroll;
 
 // The 8 codes of a lane as one bit field, code j in bits NB*j .. NB*j+NB-1. `tile_codes`
@@ -254,7 +257,11 @@ __device__ __forceinline__ float code_magic(uint64_t field, int j) {
   }
 }
 
-template <int NB, int OUT_DT, int MAXB>
+// META 1: scale and zero both second-level 8-bit codes in runs of a power-of-two length (the
+// quant_scale + quant_zero layout): the tile's code and run bases are formed once and a chunk's
+// group and run are 32-bit offsets from them (the per-chunk 64-bit index work and the meta-kind
+// branches were most of this kernel's integer instructions, which bound it). META 0: any meta.
+template <int NB, int OUT_DT, int MAXB, int META>
 __global__ void __launch_bounds__(kDBlock) dequant_axis1_kernel(
     const __grid_constant__ DBatch<MAXB> batch) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -273,6 +280,14 @@ __global__ void __launch_bounds__(kDBlock) dequant_axis1_kernel(
     const uint32_t* words = reinterpret_cast<const uint32_t*>(a.packed) + w0;
     const int64_t g0 = e0 >> a.log2_group;
     const int lane0 = warp * (kD1Unroll * 256) + lane * 8;
+    // META 1: this tile's 8-bit codes from group g0, its runs from run g0 >> L (rem0 groups in)
+    const uint8_t* qs = static_cast<const uint8_t*>(a.scale) + g0;
+    const uint8_t* qz = static_cast<const uint8_t*>(a.zero) + g0;
+    const int L = a.log2_meta_group;
+    const int64_t run0 = META ? g0 >> L : 0;
+    const int rem0 = META ? static_cast<int>(g0 - (run0 << L)) : 0;
+    const float2* ms = reinterpret_cast<const float2*>(a.scale_mm) + run0;
+    const float2* mz = reinterpret_cast<const float2*>(a.zero_mm) + run0;
     uint64_t field[kD1Unroll];
     float sc[kD1Unroll], zr[kD1Unroll];
 #pragma unroll
@@ -280,9 +295,18 @@ __global__ void __launch_bounds__(kDBlock) dequant_axis1_kernel(
       const int li = lane0 + u * 256;
       if (li < rem) {  // n and G are multiples of 8: a lane's 8 elements share one group
         field[u] = codes8_field<NB>(tile_codes, words, r0, li);
-        const int64_t g = g0 + (li >> a.log2_group);
-        sc[u] = meta_value(a, a.scale, a.scale_mm, g);
-        zr[u] = meta_value(a, a.zero, a.zero_mm, g);
+        if constexpr (META == 1) {
+          // meta_value's arithmetic: (code - zero2) * step2 of the group's run
+          const int gi = li >> a.log2_group;
+          const int ri = (rem0 + gi) >> L;
+          const float2 s2 = __ldg(ms + ri), z2 = __ldg(mz + ri);
+          sc[u] = __fmul_rn(__fsub_rn(u2f_small(__ldg(qs + gi)), s2.y), s2.x);
+          zr[u] = __fmul_rn(__fsub_rn(u2f_small(__ldg(qz + gi)), z2.y), z2.x);
+        } else {
+          const int64_t g = g0 + (li >> a.log2_group);
+          sc[u] = meta_value(a, a.scale, a.scale_mm, g);
+          zr[u] = meta_value(a, a.zero, a.zero_mm, g);
+        }
       }
     }
 #pragma unroll
@@ -558,11 +582,18 @@ static cudaError_t launch_nb_dt(const DequantJob* jobs, int n, cudaStream_t st) 
     fill_dbatch<MAXB>(jobs, n, kDTile1, &b);
     const int64_t tiles = b.tile_start[b.n];
     if (tiles == 0) return cudaSuccess;
+    bool both_runs = b.c.log2_meta_group >= 0;  // every matrix: 8-bit scale and zero
+    for (int i = 0; i < n; ++i) both_runs = both_runs && jobs[i].scale_mm && jobs[i].zero_mm;
     int resident = 0;
-    const cudaError_t e = resident_blocks(dequant_axis1_kernel<NB, OUT_DT, MAXB>, &resident);
+    cudaError_t e = both_runs
+                        ? resident_blocks(dequant_axis1_kernel<NB, OUT_DT, MAXB, 1>, &resident)
+                        : resident_blocks(dequant_axis1_kernel<NB, OUT_DT, MAXB, 0>, &resident);
     if (e != cudaSuccess) return e;
     const int64_t blocks = tiles < resident ? tiles : resident;
-    dequant_axis1_kernel<NB, OUT_DT, MAXB><<<(unsigned)blocks, kDBlock, 0, st>>>(b);
+    if (both_runs)
+      dequant_axis1_kernel<NB, OUT_DT, MAXB, 1><<<(unsigned)blocks, kDBlock, 0, st>>>(b);
+    else
+      dequant_axis1_kernel<NB, OUT_DT, MAXB, 0><<<(unsigned)blocks, kDBlock, 0, st>>>(b);
   } else {
     if constexpr (OUT_DT != kF32 && NB != 3) {
       bool cols8 = true;

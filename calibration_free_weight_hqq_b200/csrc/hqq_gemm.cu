@@ -971,14 +971,15 @@ __global__ void __launch_bounds__(skinny::kThreads, 2)
 #ifndef HQQ_GEMV_DEPTH
 #define HQQ_GEMV_DEPTH 4
 #endif
-// When the next kernel on the stream may launch (HQQ_FLAG_OVERLAP_WEIGHTS): 1 = after this
-// kernel's last tile, 0 = at entry. At entry the dependent's persistent grid, sized for an idle
-// GPU, started partly late and its clusters then carried several tiles each (measured slower).
 // Where the next row tile's first code loads are issued: 1 = between the arrive and the wait of
 // the tile's cluster barrier, 0 = before the barrier.
 #ifndef HQQ_GEMV_SPLIT_SYNC
 #define HQQ_GEMV_SPLIT_SYNC 1
 #endif
+// When the next kernel on the stream may launch (HQQ_FLAG_OVERLAP_WEIGHTS): 1 = after this
+// kernel's last tile, 0 = at entry. At entry the dependent's persistent grid, sized for an idle
+// GPU, started partly late and its clusters then carried several tiles each (measured slower,
+// also when only the grids with one row tile per cluster triggered at entry).
 #ifndef HQQ_GEMV_TRIGGER_LATE
 #define HQQ_GEMV_TRIGGER_LATE 1
 #endif
