@@ -929,6 +929,7 @@ SINGLE_CASES = {
     "quantize_1b_g32": (16384, 8192, "bf16", 1, 32, 1),
     "quantize_3b_g64": (16384, 8192, "bf16", 3, 64, 1),
     "quantize_fp16_4096x1024": (4096, 1024, "f16", 4, 64, 1),
+    "dequantize_2b_g16_axis0": (16384, 8192, "bf16", 2, 16, 0),
 }
 # dequantize with 8-bit second-level scale/zero (runs of 128), the layouts of the 70B MLP
 # workload's two matrices, on a [16384, 8192] bf16 weight
@@ -1011,7 +1012,7 @@ def single(kind: str, reps: int = 10):
     pk, s, z = hqq.hqq_quantize(W, nbits, G, axis)
     D = torch.empty_like(W)
     run = (lambda: hqq.hqq_dequantize(pk, s, z, rows, cols, nbits, G, axis, out=D)) \
-        if kind == "dequantize" else \
+        if kind.startswith("dequantize") else \
         (lambda: hqq.hqq_quantize(W, nbits, G, axis, Wq_packed=pk, scale=s, zero=z))
     for _ in range(2):
         run()
@@ -1027,7 +1028,7 @@ def single(kind: str, reps: int = 10):
     mufu = 2 * 21 * n / (ms * 1e-3) / (MUFU_PER_CLK_PER_SM * N_SM * SM_MAX_MHZ * 1e6)
     return {"single": kind, "shape": [rows, cols], "nbits": nbits, "group_size": G,
             "axis": axis, "ms": round(ms, 4), "Gweights_per_s": round(n / ms / 1e6, 2),
-            "mufu_frac": round(mufu, 4) if kind != "dequantize" else None}
+            "mufu_frac": round(mufu, 4) if not kind.startswith("dequantize") else None}
 
 
 def main():

@@ -375,15 +375,45 @@ def exact_grid_weights(rows: int, cols: int, nbits: int, G: int, axis: int, seed
 
 def dequant_parity(rows: int, cols: int, nbits: int, G: int, axis: int, out_dtype: str,
                    meta_dtype: str = "f32", quant_meta: bool = False, meta_group: int = 128,
-                   seed: int = 0) -> None:
+                   seed: int = 0, one_sided: str | None = None) -> None:
     """hqq_dequantize_ex against the oracle's dequantize on codes, scale and zero drawn here
     (packed by the oracle; with quant_meta, 8-bit meta codes and run pairs drawn here and
-    decoded by the oracle's dequantize_meta): bit-exact after one rounding to out_dtype."""
+    decoded by the oracle's dequantize_meta): bit-exact after one rounding to out_dtype.
+    one_sided = "scale" or "zero": only that side is second-level, the other is stored in
+    meta_dtype."""
     rng = np.random.default_rng(seed)
     qmax = 2 ** nbits - 1
     ng = rows * cols // G
     codes = rng.integers(0, qmax + 1, size=rows * cols).astype(np.uint8)
     packed = torch.from_numpy(oracle.pack(codes, nbits)).cuda()
+    if one_sided is not None:
+        runs = (ng + meta_group - 1) // meta_group
+        qs = rng.integers(0, 256, size=ng).astype(np.uint8)
+        smm = np.stack([rng.random(runs) * 1e-4 + 1e-6, rng.random(runs) * 10], 1).astype(np.float32)
+        plain_s = oracle.round_to_dtype((rng.random(ng) * 0.02 + 1e-4).astype(np.float32), meta_dtype)
+        plain_z = oracle.round_to_dtype((rng.random(ng) * qmax).astype(np.float32), meta_dtype)
+        params = hqq.make_params(nbits, G, axis, w_dtype=torch.bfloat16,
+                                 meta_dtype=TORCH_OF[meta_dtype],
+                                 quant_scale=one_sided == "scale", quant_zero=one_sided == "zero",
+                                 meta_group_size=meta_group)
+        q8 = torch.from_numpy(qs).cuda()
+        mm = torch.from_numpy(smm).cuda()
+        if one_sided == "scale":
+            scale, zero = oracle.dequantize_meta(qs, smm, meta_group), plain_z
+            out = {"Wq_packed": packed, "scale": q8, "scale_mm": mm, "zero_mm": None,
+                   "zero": torch.from_numpy(plain_z).to(TORCH_OF[meta_dtype]).cuda()}
+        else:
+            scale, zero = plain_s, oracle.dequantize_meta(qs, smm, meta_group)
+            out = {"Wq_packed": packed, "zero": q8, "zero_mm": mm, "scale_mm": None,
+                   "scale": torch.from_numpy(plain_s).to(TORCH_OF[meta_dtype]).cuda()}
+        D = hqq.hqq_dequantize_ex(out, rows, cols, params, out_dtype=TORCH_OF[out_dtype])
+        torch.cuda.synchronize()
+        want = oracle.round_to_dtype(oracle.dequantize(codes, scale, zero, rows, cols, G, axis),
+                                     out_dtype)
+        got = D.float().cpu().numpy()
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), \
+            np.flatnonzero(got != want)[:8]
+        return
     params = hqq.make_params(nbits, G, axis, w_dtype=torch.bfloat16,
                              meta_dtype=TORCH_OF[meta_dtype], quant_scale=quant_meta,
                              quant_zero=quant_meta, meta_group_size=meta_group)

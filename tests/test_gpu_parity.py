@@ -241,6 +241,14 @@ def test_dequantize_bit_exact_second_level(nbits, G, axis):
                        seed=nbits + mg)
 
 
+@pytest.mark.parametrize("side", ["scale", "zero"])
+@pytest.mark.parametrize("nbits,G", [(3, 64), (1, 32), (4, 64)])
+def test_dequantize_bit_exact_one_sided_second_level(nbits, G, side):
+    # only one of scale / zero as 8-bit codes (runs of 128), the other stored in bf16
+    dequant_parity(64, 40 * G, nbits, G, 1, "bf16", meta_dtype="bf16", meta_group=128,
+                   seed=nbits * 7 + G, one_sided=side)
+
+
 @pytest.mark.parametrize("rows,cols", [(16384, 8192), (4096, 11008)])
 def test_dequantize_bit_exact_bench_layout(rows, cols):
     # 4-bit, group 64, axis 1, bf16 meta and output: the layout of the bench step (its
