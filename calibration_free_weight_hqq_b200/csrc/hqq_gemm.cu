@@ -212,8 +212,11 @@ __device__ __forceinline__ float meta_f32(uint32_t h) {
 //     multicasts its commits to both CTAs' barriers; one thread of the follower relays "our
 //     half is written" to the leader with one cluster-scope arrive per k-block.
 namespace sm2 {
-constexpr int kStagesL = 4;   // X boxes + packed codes
-constexpr int kStagesB = 3;   // dequantized half operand
+#ifndef HQQ_GEMM_STAGES_B
+#define HQQ_GEMM_STAGES_B 4
+#endif
+constexpr int kStagesL = 4;                  // X boxes + packed codes
+constexpr int kStagesB = HQQ_GEMM_STAGES_B;  // dequantized half operand
 constexpr int kDqWarps = 16;
 constexpr int kRows = kBN / 2;                                   // W' rows per CTA
 constexpr int kDqIters = kRows * (kBK / 8) / (32 * kDqWarps);   // 2
