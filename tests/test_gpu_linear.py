@@ -99,6 +99,7 @@ def test_linear_one_hot_is_bit_exact_transposed_weight():
     (777, 1032, 704, "f16", "bf16", False),
     (300, 256, 320, "bf16", "bf16", True),    # K/64 odd: one value per copy
     (260, 512, 192, "f16", "f32", False),     # K/64 odd, fp32 meta
+    (129, 136, 64, "bf16", "bf16", True),     # 2-SM kernel: one k-block, ragged M and N
 ])
 def test_linear_random_matches_oracle(M, N, K, dtype, meta, with_bias):
     codes, scale, zero, dev = make_layer(N, K, 100 + M + N + K, meta)
